@@ -1,0 +1,239 @@
+"""Plain fp64 definitions of RoPE attention, its squared-error loss and closed-form gradient.
+
+TEST INFRASTRUCTURE ONLY (see ``oracle/__init__.py``).  Shares no code with the CUDA path.
+
+Sources, by page and section:
+
+* "Technische Samenvatting: RoPE Attention kan bijna lineair worden getraind"
+  (summary of arXiv 2412.17316), section Probleemdefinitie and Methodologie 1
+  "Gradientherformulering in gesloten vorm": the loss of RoPE attention with respect
+  to the weight matrices, and the closed form dLoss/dx = A~^T vec(gamma(x)) built from
+  s(x) (the normalised softmax), l(x) (attention output minus target), beta(x) (the
+  error combined with the value matrix) and gamma(x).
+* Same page, Methodologie 2 "Low-Rank Benaderingsstrategie": gamma split into
+  gamma_1 = diag(s) beta and gamma_2 = s s^T beta, gamma = gamma_1 - gamma_2.
+* "HyperAttention" article (nearauto.com), section 方法の概要: exact attention is
+  D^-1 A V with A = exp(Q K^T) taken entrywise and D the diagonal of A's row sums.
+
+Readings where the pages are silent (each is listed in the design notes):
+
+* scores are Q~ K~^T / sqrt(d); the loss is 1/2 ||O - E||_F^2, summed over every
+  (batch, head) instance;
+* RoPE rotates the adjacent pairs (2k, 2k+1), k = 0..d/2-1, counter-clockwise by
+  phi_{i,k} = pos_i * base^(-2k/d);
+* Q = A1 WQ, K = A2 WK, V = A3 WV (row-vector convention, W[in][out]); each (b, h) is an
+  independent instance, W is per head and shared over the batch, dW sums over b;
+* the causal mask removes keys j > i by index.
+
+The method's exact result *is* the plain definition, so the oracle computes the
+definition: projections, rotation, a two-pass softmax per query row, O = s V,
+l = O - E, beta = l V^T, gamma = diag(s) beta - s s^T beta row by row, then
+dQ~ = gamma K~ / sqrt(d), dK~ = gamma^T Q~ / sqrt(d), dV = s^T l, the inverse rotation
+and dW = A^T dX.  Query rows are processed in blocks so no n x n array is held.
+"""
+from __future__ import annotations
+
+import math
+from typing import Dict, Iterable, Optional
+
+import numpy as np
+
+# Every oracle function has a pin in tests/test_oracle.py; none is unpinned.
+ORACLE_PARITY_PINNED = True
+
+F64 = np.float64
+
+
+def rope_theta(d: int, base: float) -> np.ndarray:
+    """theta_k = base^(-2k/d), k = 0 .. d/2-1, in fp64."""
+    k = np.arange(d // 2, dtype=F64)
+    return np.power(F64(base), -2.0 * k / F64(d))
+
+
+def rope_angles(pos: np.ndarray, d: int, base: float) -> np.ndarray:
+    """phi[i, k] = pos_i * theta_k (fp64), shape [n][d/2]."""
+    return np.asarray(pos, dtype=F64)[:, None] * rope_theta(d, base)[None, :]
+
+
+def rope_rotate(X: np.ndarray, phi: np.ndarray) -> np.ndarray:
+    """Rotate each pair (x_2k, x_2k+1) of every row of X [n][d] by the angle phi[i, k].
+
+    (x_2k, x_2k+1) -> (x_2k cos phi - x_2k+1 sin phi, x_2k sin phi + x_2k+1 cos phi).
+    The inverse rotation is ``rope_rotate(X, -phi)``.
+    """
+    X = np.asarray(X, dtype=F64)
+    c, s = np.cos(phi), np.sin(phi)
+    x0, x1 = X[:, 0::2], X[:, 1::2]
+    out = np.empty_like(X)
+    out[:, 0::2] = x0 * c - x1 * s
+    out[:, 1::2] = x0 * s + x1 * c
+    return out
+
+
+def softmax_rows(Z: np.ndarray):
+    """Two-pass softmax along each row: s = exp(Z - max) / sum; also returns log-sum-exp.
+
+    Entries equal to -inf (masked keys) get probability 0.
+    """
+    m = np.max(Z, axis=1, keepdims=True)
+    e = np.exp(Z - m)
+    tot = np.sum(e, axis=1, keepdims=True)
+    s = e / tot
+    lse = (m + np.log(tot))[:, 0]
+    return s, lse
+
+
+def gamma_closed_form(s: np.ndarray, beta: np.ndarray) -> np.ndarray:
+    """gamma = gamma_1 - gamma_2 with gamma_1 = diag(s) beta and gamma_2 = s s^T beta, per row.
+
+    For row i (one query): gamma_1,i = s_i o beta_i and gamma_2,i = s_i (s_i^T beta_i).
+    """
+    gamma_1 = s * beta
+    gamma_2 = s * np.sum(s * beta, axis=1, keepdims=True)
+    return gamma_1 - gamma_2
+
+
+def scores_rows(Qt: np.ndarray, Kt: np.ndarray, rows: np.ndarray, causal: bool) -> np.ndarray:
+    """Z[r, j] = Q~_{rows[r]} . K~_j / sqrt(d), with keys j > rows[r] set to -inf if causal."""
+    d = Qt.shape[1]
+    Z = (Qt[rows] @ Kt.T) / math.sqrt(d)
+    if causal:
+        j = np.arange(Kt.shape[0])
+        Z = np.where(j[None, :] > np.asarray(rows)[:, None], -np.inf, Z)
+    return Z
+
+
+def _project(A1, A2, A3, WQ, WK, WV, pos, base):
+    d = WQ.shape[0]
+    phi = rope_angles(pos, d, base)
+    Q = np.asarray(A1, F64) @ np.asarray(WQ, F64)
+    K = np.asarray(A2, F64) @ np.asarray(WK, F64)
+    V = np.asarray(A3, F64) @ np.asarray(WV, F64)
+    return rope_rotate(Q, phi), rope_rotate(K, phi), V, phi
+
+
+def instance_forward_backward(A1, A2, A3, E, WQ, WK, WV, pos, causal: bool, base: float,
+                              want_grad: bool = True, rb: int = 256) -> Dict[str, np.ndarray]:
+    """One (batch, head) instance: forward, loss and (optionally) the closed-form gradient.
+
+    Inputs are [n][d] (A1, A2, A3, E) and [d][d] (WQ, WK, WV).  Returns O, lse, loss and,
+    with ``want_grad``, dQt, dKt, dV (gradients w.r.t. the rotated Q~, K~ and V),
+    dQ, dK (un-rotated) and dWQ, dWK, dWV.
+    """
+    n, d = np.shape(A1)
+    c = 1.0 / math.sqrt(d)
+    Qt, Kt, V, phi = _project(A1, A2, A3, WQ, WK, WV, pos, base)
+    E = np.asarray(E, F64)
+    O = np.empty((n, d), F64)
+    lse = np.empty(n, F64)
+    loss = 0.0
+    if want_grad:
+        dQt = np.empty((n, d), F64)
+        dKt = np.zeros((n, d), F64)
+        dV = np.zeros((n, d), F64)
+    for r0 in range(0, n, rb):
+        r1 = min(n, r0 + rb)
+        rows = np.arange(r0, r1)
+        # causal: every key beyond the block's last row is masked for all its rows
+        kend = r1 if causal else n
+        Z = scores_rows(Qt, Kt[:kend], rows, causal)
+        s, lse[r0:r1] = softmax_rows(Z)                  # s(x)
+        O[r0:r1] = s @ V[:kend]                          # O = s V
+        ell = O[r0:r1] - E[r0:r1]                        # l(x) = O - E
+        loss += 0.5 * float(np.sum(ell * ell))
+        if not want_grad:
+            continue
+        beta = ell @ V[:kend].T                          # beta(x) = l V^T
+        gamma = gamma_closed_form(s, beta)               # gamma = diag(s)beta - s s^T beta
+        dQt[r0:r1] = (gamma @ Kt[:kend]) * c
+        dKt[:kend] += (gamma.T @ Qt[r0:r1]) * c
+        dV[:kend] += s.T @ ell
+    out = {"O": O, "lse": lse, "loss": loss, "Qt": Qt, "Kt": Kt, "V": V}
+    if want_grad:
+        dQ = rope_rotate(dQt, -phi)
+        dK = rope_rotate(dKt, -phi)
+        out.update(dQt=dQt, dKt=dKt, dV=dV, dQ=dQ, dK=dK,
+                   dWQ=np.asarray(A1, F64).T @ dQ,
+                   dWK=np.asarray(A2, F64).T @ dK,
+                   dWV=np.asarray(A3, F64).T @ dV)
+    return out
+
+
+def instance_loss(A1, A2, A3, E, WQ, WK, WV, pos, causal: bool, base: float) -> float:
+    """Loss = 1/2 ||O - E||_F^2 of one instance (forward only)."""
+    return instance_forward_backward(A1, A2, A3, E, WQ, WK, WV, pos, causal, base,
+                                     want_grad=False)["loss"]
+
+
+def _heads(inp, heads: Optional[Iterable[int]]):
+    H = inp["WQ"].shape[0]
+    return range(H) if heads is None else list(heads)
+
+
+def forward_backward(inp: Dict[str, np.ndarray], causal: bool, base: float,
+                     heads: Optional[Iterable[int]] = None,
+                     want_grad: bool = True) -> Dict[str, np.ndarray]:
+    """All (b, h) instances of a batch; ``heads`` restricts the work to some heads.
+
+    Returns O [B][H][n][d], lse [B][H][n], loss (sum over the instances computed) and
+    dWQ, dWK, dWV [H][d][d] (summed over b).  Entries of heads not computed are NaN.
+    """
+    B, H, n, d = inp["A1"].shape
+    O = np.full((B, H, n, d), np.nan)
+    lse = np.full((B, H, n), np.nan)
+    dW = {k: np.full((H, d, d), np.nan) for k in ("dWQ", "dWK", "dWV")}
+    extra = {k: np.full((B, H, n, d), np.nan) for k in ("dQt", "dKt", "dV")} if want_grad else {}
+    loss = 0.0
+    for h in _heads(inp, heads):
+        if want_grad:
+            for k in dW:
+                dW[k][h] = 0.0
+        for b in range(B):
+            r = instance_forward_backward(inp["A1"][b, h], inp["A2"][b, h], inp["A3"][b, h],
+                                          inp["E"][b, h], inp["WQ"][h], inp["WK"][h],
+                                          inp["WV"][h], inp["pos"], causal, base, want_grad)
+            O[b, h], lse[b, h] = r["O"], r["lse"]
+            loss += r["loss"]
+            if want_grad:
+                for k in dW:
+                    dW[k][h] += r[k]
+                for k in extra:
+                    extra[k][b, h] = r[k]
+    out = {"O": O, "lse": lse, "loss": loss}
+    if want_grad:
+        out.update(dW)
+        out.update(extra)
+    return out
+
+
+def loss_only(inp, causal, base) -> float:
+    return forward_backward(inp, causal, base, want_grad=False)["loss"]
+
+
+def forward_rows(inp: Dict[str, np.ndarray], b: int, h: int, rows, causal: bool,
+                 base: float) -> Dict[str, np.ndarray]:
+    """O, lse, and the gradient rows dQ~ for selected query rows of instance (b, h).
+
+    Row i needs only Q~_i and all of K~ and V, so sampled rows of a large instance
+    cost O(n d) each.  dQ~_i = gamma_i K~ / sqrt(d) with gamma_i from s_i and
+    beta_i = l_i V^T.
+    """
+    rows = np.asarray(rows)
+    A1, A2, A3, E = (inp[k][b, h] for k in ("A1", "A2", "A3", "E"))
+    d = A1.shape[1]
+    phi_r = rope_angles(np.asarray(inp["pos"])[rows], d, base)
+    Qt_r = rope_rotate(np.asarray(A1, F64)[rows] @ np.asarray(inp["WQ"][h], F64), phi_r)
+    Kt = rope_rotate(np.asarray(A2, F64) @ np.asarray(inp["WK"][h], F64),
+                     rope_angles(inp["pos"], d, base))
+    V = np.asarray(A3, F64) @ np.asarray(inp["WV"][h], F64)
+    Z = (Qt_r @ Kt.T) / math.sqrt(d)
+    if causal:
+        j = np.arange(Kt.shape[0])
+        Z = np.where(j[None, :] > rows[:, None], -np.inf, Z)
+    s, lse = softmax_rows(Z)
+    O = s @ V
+    ell = O - np.asarray(E, F64)[rows]
+    beta = ell @ V.T
+    gamma = gamma_closed_form(s, beta)
+    dQt = (gamma @ Kt) / math.sqrt(d)
+    return {"O": O, "lse": lse, "dQt": dQt}
