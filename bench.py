@@ -1,0 +1,431 @@
+#!/usr/bin/env python
+"""Throughput of the exact RoPE-attention loss + closed-form gradient (forward + backward).
+
+One step = rope_attn_fwd (with the loss) followed by rope_attn_loss_bwd reusing the
+forward's workspace, over one batch of the workload: every step of the hot path
+(RoPE table, projections + RoPE, attention forward with the loss epilogue, the
+tile-wise closed-form backward, inverse RoPE + weight gradients, loss reduction).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME]
+
+With N > 1 it is launched by torch.distributed.run, one process per GPU; every rank runs
+its own copy of the workload (the (batch, head) instances are independent, so the work
+shards with no collective on the data path) and the reported value is the work of all
+ranks divided by the slowest rank's device time.  Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from workloads import WORKLOADS, flop_count, make_inputs, pair_count  # noqa: E402
+
+DEFAULT_WORKLOAD = "b2_h32_n8192_d128_bf16_causal"
+METRIC = "RoPE-attention loss+grad fwd+bwd TFLOP/s, % of B200 BF16 tensor peak"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                  "sm_max_mhz": 1965.0}
+L2_BYTES = 126 * 2 ** 20
+# B200: 148 SMs x 128 fp32 lanes x 2 flop per FMA at the maximum SM clock
+FP32_SIMT_LANES = 148 * 128
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=list(WORKLOADS))
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def workload_config(w, n_gpus):
+    return {"workload": w.name, "B": w.B, "H": w.H, "n": w.n, "d": w.d, "dtype": w.dtype,
+            "causal": w.causal, "rope_base": w.rope_base, "global_batch": w.B * n_gpus,
+            "seq_len": w.n, "parallelism": f"replicas{n_gpus}" if n_gpus > 1 else "single",
+            "l2": "inputs larger than L2 (%.0f MB of inputs per step vs 126 MB L2)"
+                  % (4 * w.B * w.H * w.n * w.d * (2 if w.dtype == "bf16" else 4) / 1e6)}
+
+
+# ---------------------------------------------------------------------------------------
+# clocks sampled with nvidia-smi during the timed region
+# ---------------------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.out = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+
+    def start(self):
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+               "-lms", "100"]
+        if self.gpu_id is not None:
+            cmd += ["-i", str(self.gpu_id)]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=self.out, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.2)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.out.flush()
+        self.out.seek(0)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.out:
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        os.unlink(self.out.name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        hi = [x for x in sm if x > 0.5 * max(sm)] or sm
+        return {"sm_mhz": statistics.median(hi), "sm_max_mhz": max(smax),
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+def _gpu_uuid(dev):
+    import torch
+    try:
+        u = torch.cuda.get_device_properties(dev).uuid
+        return "GPU-" + str(u)
+    except Exception:
+        return None
+
+
+# ---------------------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------------------
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    from loss_closed_form_b200 import rope_attn as ra
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    w = WORKLOADS[args.workload]
+    inp = make_inputs(w, seed=w.seed + rank)
+    tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    host = {k: torch.from_numpy(inp[k]).to(tdt).pin_memory()
+            for k in ("A1", "A2", "A3", "E", "WQ", "WK", "WV")}
+    host["pos"] = torch.from_numpy(inp["pos"]).pin_memory()
+    del inp
+    t = {k: v.to(dev) for k, v in host.items()}
+    m = ra.RopeAttention(t["A1"], t["A2"], t["A3"], t["WQ"], t["WK"], t["WV"], t["E"],
+                         t["pos"], w.causal, w.rope_base)
+    stream = torch.cuda.current_stream(dev)
+    flops = flop_count(w)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(max(3, args.warmup)):
+        m.step()
+    torch.cuda.synchronize(dev)
+    st = ra.last_error()
+    if st != ra.RA_OK:
+        raise RuntimeError(f"kernel status after warm-up: {ra.status_string(st)}")
+
+    # ---- device-timed region: inputs resident in HBM -------------------------------------
+    clocks = ClockSampler(_gpu_uuid(dev)) if rank == 0 else None
+    if clocks:
+        clocks.start()
+    ra.launch_count()
+    ra.profile_read()
+    ra.profile_enable(True)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize(dev)
+    e0.record(stream)
+    for _ in range(args.steps):
+        m.step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    launches = ra.launch_count()
+    per_kernel = ra.profile_read()
+    ra.profile_enable(False)
+    clk = clocks.stop() if clocks else None
+    ms = e0.elapsed_time(e1)
+    st = ra.last_error()
+    if st != ra.RA_OK:
+        raise RuntimeError(f"kernel status after timing: {ra.status_string(st)}")
+    ms_max = ms
+    if world > 1:
+        x = torch.tensor([ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(x, op=dist.ReduceOp.MAX)
+        ms_max = float(x.item())
+
+    # ---- end to end: pinned host inputs -> device, step, loss + dW back to the host -----
+    e2e = None
+    if not args.no_e2e:
+        out_host = {"loss": torch.empty((), dtype=torch.float32).pin_memory(),
+                    "dWQ": torch.empty_like(m.dWQ, device="cpu").pin_memory(),
+                    "dWK": torch.empty_like(m.dWK, device="cpu").pin_memory(),
+                    "dWV": torch.empty_like(m.dWV, device="cpu").pin_memory()}
+        h2d = sum(v.numel() * v.element_size() for v in host.values())
+        d2h = sum(v.numel() * v.element_size() for v in out_host.values())
+
+        def e2e_step():
+            for k, v in host.items():
+                t[k].copy_(v, non_blocking=True)
+            m.step()
+            out_host["loss"].copy_(m.loss, non_blocking=True)
+            out_host["dWQ"].copy_(m.dWQ, non_blocking=True)
+            out_host["dWK"].copy_(m.dWK, non_blocking=True)
+            out_host["dWV"].copy_(m.dWV, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize(dev)
+        barrier()
+        torch.cuda.synchronize(dev)
+        e0.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier()
+        ms_e2e = e0.elapsed_time(e1)
+        if world > 1:
+            x = torch.tensor([ms_e2e], dtype=torch.float64, device=dev)
+            dist.all_reduce(x, op=dist.ReduceOp.MAX)
+            ms_e2e = float(x.item())
+        if not math.isfinite(float(out_host["loss"])):
+            raise RuntimeError("non-finite loss in the end-to-end run")
+        e2e = {"value": round(world * flops * args.steps / (ms_e2e * 1e-3) / 1e12, 3),
+               "unit": "TFLOP/s", "ms_per_step": round(ms_e2e / args.steps, 4),
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+
+    if rank != 0:
+        return None
+
+    # ---- roofline of the dominant kernel ------------------------------------------------
+    pk, src = peaks()
+    top = max(per_kernel.items(), key=lambda kv: kv[1][0])
+    top_name, (top_ms, top_n) = top
+    avg_ms = top_ms / max(1, top_n)
+    roof = roofline(w, top_name, avg_ms, pk, src)
+    value = world * flops * args.steps / (ms_max * 1e-3) / 1e12
+    total_kernel_ms = sum(v[0] for v in per_kernel.values())
+    line = {
+        "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": max(3, args.warmup),
+        "ms_per_step": round(ms_max / args.steps, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+        "config": workload_config(w, world),
+        "frac_of_bf16_peak": round(value / world / pk["bf16_tflops"], 4),
+        "tokens_per_s": round(world * w.B * w.n * args.steps / (ms_max * 1e-3), 1),
+        "roofline": roof,
+        "kernels": {k: {"ms_per_step": round(v[0] / args.steps, 4),
+                        "launches": v[1], "share": round(v[0] / total_kernel_ms, 4)}
+                    for k, v in sorted(per_kernel.items(), key=lambda kv: -kv[1][0])},
+        "gpu_launches": int(launches),
+        "clocks": clk,
+        "e2e": e2e,
+        "peaks_source": src,
+    }
+    return line
+
+
+def roofline(w, kname, avg_ms, pk, src):
+    """Algorithmic work of one launch of the dominant kernel over its measured duration."""
+    BH = w.B * w.H
+    P = pair_count(w.n, w.causal)
+    d, n = w.d, w.n
+    tensor_kernels = {"attn_bwd_tc": 10.0 * d * P * BH, "attn_fwd_tc": 4.0 * d * P * BH}
+    simt_kernels = {"attn_bwd_simt": 10.0 * d * P * BH, "attn_fwd_simt": 4.0 * d * P * BH,
+                    "proj_rope_simt": 6.0 * n * d * d * BH, "dw_partial_simt": 6.0 * n * d * d * BH}
+    traffic = measured_traffic(kname)
+    if kname in tensor_kernels:
+        flop = tensor_kernels[kname]
+        peak = pk["bf16_tflops"]
+        ach = flop / (avg_ms * 1e-3) / 1e12
+        return {"kernel": kname, "bound": "tensor", "achieved": round(ach, 3), "peak": peak,
+                "unit": "TFLOP/s", "frac": round(ach / peak, 4), "traffic": traffic,
+                "peak_source": f"{src} bf16 dense (burst)",
+                "algorithmic_per_launch": flop, "avg_launch_ms": round(avg_ms, 4)}
+    if kname in simt_kernels:
+        flop = simt_kernels[kname]
+        peak = FP32_SIMT_LANES * 2 * pk.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
+        ach = flop / (avg_ms * 1e-3) / 1e12
+        return {"kernel": kname, "bound": "alu", "achieved": round(ach, 3),
+                "peak": round(peak, 2), "unit": "TFLOP/s", "frac": round(ach / peak, 4),
+                "traffic": traffic,
+                "peak_source": "fp32 FMA: 148 SMs x 128 lanes x 2 flop x max SM clock",
+                "algorithmic_per_launch": flop, "avg_launch_ms": round(avg_ms, 4)}
+    # memory-bound kernels: algorithmic bytes are not modelled here
+    return {"kernel": kname, "bound": "hbm", "achieved": None, "peak": pk["hbm_gbs"],
+            "unit": "GB/s", "frac": None, "traffic": traffic, "avg_launch_ms": round(avg_ms, 4)}
+
+
+def measured_traffic(kname):
+    """DRAM bytes per launch from a committed ncu summary, if it matches the current source."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+    except (OSError, ValueError):
+        return None
+    ent = rec.get(kname)
+    if not ent:
+        return None
+    if ent.get("source_sha") != kernel_source_sha():
+        return None
+    return ent.get("dram_bytes_per_launch")
+
+
+def kernel_source_sha():
+    import hashlib
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "loss_closed_form_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        if f.endswith((".cu", ".cuh")):
+            with open(os.path.join(csrc, f), "rb") as fh:
+                h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+# ---------------------------------------------------------------------------------------
+# the fp64 oracle on the host cores (reference arm and CPU baseline)
+# ---------------------------------------------------------------------------------------
+def oracle_sample_time(w, instances, seed=0):
+    """Run the oracle on `instances` (b, h) instances of workload w; return (seconds, flops)."""
+    import oracle
+    one = w.with_sizes(B=1, H=1)
+    inp = make_inputs(one, seed=seed)
+    t0 = time.perf_counter()
+    for _ in range(instances):
+        oracle.forward_backward(inp, w.causal, w.rope_base)
+    dt = time.perf_counter() - t0
+    return dt, flop_count(one) * instances
+
+
+def host_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count()
+
+
+def cpu_baseline(w, budget_s=12.0):
+    dt, fl = oracle_sample_time(w, 1)
+    k = max(1, min(64, int(budget_s / max(dt, 1e-3))))
+    if k > 1:
+        dt2, fl2 = oracle_sample_time(w, k)
+        dt, fl, inst = dt + dt2, fl + fl2, k + 1
+    else:
+        inst = 1
+    return {"value": round(fl / dt / 1e12, 6), "unit": "TFLOP/s", "cores": host_cores(),
+            "kind": "oracle",
+            "sample": f"{inst} (b,h) instance(s) of {w.name} (n={w.n}, d={w.d}, "
+                      f"causal={w.causal}), fp64 NumPy, {dt:.1f} s"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    w = WORKLOADS[args.workload]
+    one = w.with_sizes(B=1, H=1)
+    # each step: the oracle on a bounded sample of the workload (whole (b,h) instances)
+    dt1, _ = oracle_sample_time(w, 1)
+    per_step = max(1, min(4, int(4.0 / max(dt1, 1e-3))))
+    import oracle
+    inp = make_inputs(one)
+    times = []
+    for i in range(max(3, args.warmup) + args.steps):
+        t0 = time.perf_counter()
+        for _ in range(per_step):
+            oracle.forward_backward(inp, w.causal, w.rope_base)
+        if i >= max(3, args.warmup):
+            times.append(time.perf_counter() - t0)
+    fl = flop_count(one) * per_step
+    total = sum(times)
+    value = fl * len(times) / total / 1e12
+    sample = (f"{per_step} (b,h) instance(s) of {w.name} per step (n={w.n}, d={w.d}, "
+              f"causal={w.causal}), fp64 NumPy oracle")
+    return {"metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": max(3, args.warmup),
+            "ms_per_step": round(1e3 * total / len(times), 2), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": workload_config(w, world), "impl": "reference",
+            "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": host_cores(),
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        line = run_reference(args, rank, world)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        line = run_ours(args, rank, world, local_rank)
+        if line is not None and world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(WORKLOADS[args.workload])
+        if line is not None:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

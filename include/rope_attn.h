@@ -1,0 +1,149 @@
+/*
+ * rope_attn.h - C ABI of librope_attn: exact RoPE softmax attention, its squared-error
+ * loss and the closed-form gradient with respect to the three weight matrices, on one
+ * NVIDIA B200 (sm_100a).
+ *
+ * What is computed (per batch b and head h, every (b, h) an independent instance):
+ *
+ *   Q~ = rot(A1 WQ),  K~ = rot(A2 WK),  V = A3 WV            (row-vector convention)
+ *   s  = softmax(Q~ K~^T / sqrt(d))   (row-wise; keys j > i masked when causal)
+ *   O  = s V,   l = O - E,   Loss = 1/2 sum_{b,h} ||O - E||_F^2
+ *   beta  = l V^T,  gamma = diag(s) beta - s s^T beta
+ *         (row-wise gamma_i = s_i o (beta_i - <l_i, O_i>))
+ *   dQ~ = gamma K~ / sqrt(d),  dK~ = gamma^T Q~ / sqrt(d),  dV = s^T l
+ *   dWQ_h = sum_b A1^T rot^-1(dQ~),  dWK_h = sum_b A2^T rot^-1(dK~),  dWV_h = sum_b A3^T dV
+ *
+ * rot() turns each adjacent pair (x_2k, x_2k+1) of row i counter-clockwise by the angle
+ * pos_i * base^(-2k/d), k = 0 .. d/2-1.
+ *
+ * Sources: "RoPE Attention kan bijna lineair worden getraind" (summary of arXiv
+ * 2412.17316), sections Probleemdefinitie and Methodologie 1 (closed-form gradient
+ * dLoss/dx = A~^T vec(gamma(x)) built from s, l, beta, gamma) and Methodologie 2
+ * (gamma_1 = diag(s) beta, gamma_2 = s s^T beta); "HyperAttention" article, section
+ * 方法の概要 (exact attention D^-1 A V with A = exp(Q K^T) entrywise).
+ *
+ * Conventions for every entry point:
+ *   - The caller owns all memory.  The library never allocates, frees or synchronises
+ *     (except rope_attn_last_error, which synchronises the given stream).
+ *   - Device pointers must be 16-byte aligned and point to contiguous arrays.
+ *   - Arguments are validated before anything is launched; a status other than RA_OK
+ *     means nothing was enqueued.  RA_ERR_CUDA means a launch failed.
+ *   - Work is enqueued asynchronously on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream) on the current CUDA device.
+ *   - A kernel that waits on an on-chip barrier gives up after a bounded time, records a
+ *     timeout in a device-side status word and returns; rope_attn_last_error reports it.
+ */
+#ifndef ROPE_ATTN_H
+#define ROPE_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  RA_OK = 0,
+  RA_ERR_INVALID_ARG = 1,   /* null pointer, bad size or flag                          */
+  RA_ERR_UNSUPPORTED = 2,   /* valid request the library does not implement (d)        */
+  RA_ERR_ALIGNMENT = 3,     /* a device pointer is not 16-byte aligned                 */
+  RA_ERR_WORKSPACE = 4,     /* workspace missing or smaller than rope_attn_workspace_bytes */
+  RA_ERR_CUDA = 5,          /* a CUDA launch or runtime call failed                    */
+  RA_ERR_TIMEOUT = 6        /* a kernel gave up waiting on an on-chip barrier          */
+} ra_status;
+
+typedef enum {
+  RA_F32 = 0,   /* fp32 I/O, fp32 arithmetic on the CUDA cores                          */
+  RA_BF16 = 1   /* bf16 I/O, bf16 tensor-core products with fp32 accumulation           */
+} ra_dtype;
+
+/* One problem: B x H independent instances of n tokens with head dimension d. */
+typedef struct {
+  int32_t B, H, n, d;      /* B, H, n >= 1; d in {64, 128}                                */
+  int32_t dtype;           /* ra_dtype: element type of A1, A2, A3, E, WQ, WK, WV and O   */
+  int32_t causal;          /* 0 or 1: mask keys j > i (by index)                          */
+  double rope_base;        /* RoPE base, > 0 (10000, 500000, ...)                         */
+  const int32_t* pos;      /* device [n] positions shared by all (b, h); NULL = 0..n-1    */
+  const void* A1;          /* device [B][H][n][d]: input of the query projection          */
+  const void* A2;          /* device [B][H][n][d]: input of the key projection            */
+  const void* A3;          /* device [B][H][n][d]: input of the value projection          */
+  const void* WQ;          /* device [H][d][d]: W[in][out], Q = A1 . WQ                   */
+  const void* WK;          /* device [H][d][d]                                            */
+  const void* WV;          /* device [H][d][d]                                            */
+  const void* E;           /* device [B][H][n][d]: target; may be NULL in rope_attn_fwd   */
+} ra_problem;
+
+/*
+ * Bytes of device workspace that rope_attn_fwd and rope_attn_loss_bwd need for `p`
+ * (0 if `p` is invalid).  The same workspace may serve both calls.
+ */
+size_t rope_attn_workspace_bytes(const ra_problem* p);
+
+/*
+ * Forward pass and loss.
+ *   O    : device [B][H][n][d], element type p->dtype (written)
+ *   lse  : device [B][H][n] fp32, natural-log log-sum-exp of each scaled score row (written)
+ *   loss : device fp32 scalar, 1/2 ||O - E||_F^2 over all instances (written); must be NULL
+ *          when p->E is NULL
+ *   ws   : device workspace of at least rope_attn_workspace_bytes(p) bytes
+ * When p->E is given, the workspace also keeps Q~, K~, V, l and <l_i, O_i> for a following
+ * rope_attn_loss_bwd(..., ws_holds_fwd = 1).
+ */
+ra_status rope_attn_fwd(const ra_problem* p, void* O, float* lse, float* loss,
+                        void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Closed-form backward: the weight gradients of Loss = 1/2 ||O - E||_F^2.
+ *   O, lse       : device, as written by rope_attn_fwd for the same problem (read)
+ *   loss         : device fp32 scalar (written; may be NULL)
+ *   dWQ/dWK/dWV  : device [H][d][d] fp32 (overwritten), summed over the batch
+ *   ws_holds_fwd : 1 if `ws` is the workspace of the immediately preceding rope_attn_fwd on
+ *                  the same problem and inputs (with E): the projections and l are reused
+ *                  instead of recomputed.  0 recomputes everything from the inputs.
+ * p->E must not be NULL.
+ */
+ra_status rope_attn_loss_bwd(const ra_problem* p, const void* O, const float* lse,
+                             float* loss, float* dWQ, float* dWK, float* dWV,
+                             void* ws, size_t ws_bytes, int32_t ws_holds_fwd, void* stream);
+
+/*
+ * Synchronises `stream`, then reports and clears the device-side status word of the current
+ * device: RA_ERR_TIMEOUT if a kernel gave up waiting since the last call, else RA_OK
+ * (RA_ERR_CUDA if the synchronisation itself failed).
+ */
+ra_status rope_attn_last_error(void* stream);
+
+/* Static, human-readable name of a status code. */
+const char* rope_attn_status_string(ra_status s);
+
+/*
+ * Number of kernel launches the library enqueued on this host thread since the last call
+ * (then reset to 0).  Used to count the launches inside a timed region.
+ */
+int64_t rope_attn_launch_count(void);
+
+/*
+ * Per-kernel timing for measurement tools.  While enabled (on != 0), every launch made by
+ * this host thread is bracketed by two CUDA events recorded on the launching stream; the
+ * events are created on first use and kept for reuse (host-side driver objects, no device
+ * memory).  Disabling drops records not yet read.
+ */
+void rope_attn_profile_enable(int32_t on);
+
+/*
+ * Waits for the recorded events, then writes for each kernel id k < max_kernels the summed
+ * device time in milliseconds (ms[k]) and the number of launches (launches[k]) since the
+ * last read, and clears the records.  Returns the number of kernel ids (see
+ * rope_attn_kernel_name), or -1 if an event query failed.
+ */
+int32_t rope_attn_profile_read(float* ms, int32_t* launches, int32_t max_kernels);
+
+/* Static name of kernel id `id` (NULL if out of range). */
+const char* rope_attn_kernel_name(int32_t id);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ROPE_ATTN_H */

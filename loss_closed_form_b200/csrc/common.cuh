@@ -1,0 +1,44 @@
+// Device helpers shared by every kernel of librope_attn.
+#pragma once
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+namespace ra {
+
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+
+__device__ __forceinline__ float to_f(float x) { return x; }
+__device__ __forceinline__ float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+template <class T> __device__ __forceinline__ T from_f(float x);
+template <> __device__ __forceinline__ float from_f<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float x) {
+  return __float2bfloat16_rn(x);
+}
+
+// Device-side status word of this library (one per device that loads it): kernels that
+// give up waiting set a nonzero code; rope_attn_last_error reads and clears it.  The whole
+// library is one translation unit, so the definition lives here.
+__device__ int g_status = 0;
+
+enum DeviceStatus : int {
+  kDevOk = 0,
+  kDevTimeout = 1,
+};
+
+__device__ __forceinline__ void flag_error(int code) { atomicMax(&g_status, code); }
+
+// Row-major [rows][cols] float tile loader with a padded smem stride.
+// Rows at or beyond `valid_rows` are filled with zeros.
+template <class T>
+__device__ __forceinline__ void load_tile_f32(float* dst, int ld_dst, const T* src, int rows,
+                                              int cols, int valid_rows, int tid, int nthr) {
+  for (int e = tid; e < rows * cols; e += nthr) {
+    int r = e / cols, c = e - r * cols;
+    dst[r * ld_dst + c] = (r < valid_rows) ? to_f(src[(size_t)r * cols + c]) : 0.f;
+  }
+}
+
+}  // namespace ra

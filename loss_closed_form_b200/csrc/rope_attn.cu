@@ -1,0 +1,387 @@
+// librope_attn: host side of the C ABI declared in include/rope_attn.h.
+//
+// Validates every argument before enqueuing anything, carves the caller's workspace,
+// and launches the kernels on the caller's stream.  Never allocates, frees or
+// synchronises (rope_attn_last_error excepted).
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#include <vector>
+
+#include "../../include/rope_attn.h"
+#include "common.cuh"
+#include "simt_kernels.cuh"
+
+namespace {
+
+thread_local int64_t t_launches = 0;
+
+// Kernel ids for launch counting and per-kernel event timing.
+enum KernelId : int {
+  K_ROPE_TABLE = 0,
+  K_PROJ_SIMT,
+  K_FWD_SIMT,
+  K_BWD_PRE,
+  K_BWD_SIMT,
+  K_DW_PART_SIMT,
+  K_DW_REDUCE,
+  K_LOSS,
+  K_COUNT
+};
+const char* const kKernelNames[K_COUNT] = {
+    "rope_table", "proj_rope_simt", "attn_fwd_simt", "bwd_pre",
+    "attn_bwd_simt", "dw_partial_simt", "dw_reduce", "loss_finalize"};
+
+struct ProfRecord {
+  int id;
+  cudaEvent_t start, stop;
+};
+struct Profiler {
+  bool on = false;
+  std::vector<ProfRecord> recs;
+  std::vector<cudaEvent_t> pool;
+  cudaEvent_t get() {
+    if (!pool.empty()) {
+      cudaEvent_t e = pool.back();
+      pool.pop_back();
+      return e;
+    }
+    cudaEvent_t e = nullptr;
+    cudaEventCreate(&e);
+    return e;
+  }
+  void recycle() {
+    for (auto& r : recs) {
+      pool.push_back(r.start);
+      pool.push_back(r.stop);
+    }
+    recs.clear();
+  }
+};
+thread_local Profiler t_prof;
+
+// Brackets one kernel launch: counts it and, when profiling, records events around it.
+struct Launch {
+  cudaStream_t st;
+  int slot = -1;
+  Launch(KernelId id, cudaStream_t s) : st(s) {
+    ++t_launches;
+    if (t_prof.on) {
+      ProfRecord r{id, t_prof.get(), t_prof.get()};
+      cudaEventRecord(r.start, st);
+      t_prof.recs.push_back(r);
+      slot = (int)t_prof.recs.size() - 1;
+    }
+  }
+  ~Launch() {
+    if (slot >= 0) cudaEventRecord(t_prof.recs[slot].stop, st);
+  }
+};
+
+constexpr size_t kAlignWs = 256;
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Workspace layout.  Offsets are bytes from the workspace base, each 256-byte aligned.
+struct Layout {
+  size_t rope;       // float2 [n][d/2]
+  size_t qt, kt, v;  // intermediate [B][H][n][d] (element size `inter`)
+  size_t ell;        // intermediate [B][H][n][d]
+  size_t delta;      // float [B][H][n]
+  size_t dqt;        // float [B][H][n][d]
+  size_t dkt;        // float [B][H][n][d]
+  size_t dv;         // float [B][H][n][d]
+  size_t dw_part;    // float [3][H][nsplit][d][d]
+  size_t loss_part;  // double [nparts]
+  size_t total;
+  int inter;         // bytes per intermediate element
+  int nsplit;        // weight-gradient row splits per head
+  int chunk;         // rows per split
+  int nparts;        // loss partial sums
+};
+
+bool is_aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
+
+ra_status check_problem(const ra_problem* p) {
+  if (!p) return RA_ERR_INVALID_ARG;
+  if (p->B < 1 || p->H < 1 || p->n < 1 || p->d < 1) return RA_ERR_INVALID_ARG;
+  if (p->dtype != RA_F32 && p->dtype != RA_BF16) return RA_ERR_INVALID_ARG;
+  if (p->causal != 0 && p->causal != 1) return RA_ERR_INVALID_ARG;
+  if (!(p->rope_base > 0.0) || !isfinite(p->rope_base)) return RA_ERR_INVALID_ARG;
+  if (!p->A1 || !p->A2 || !p->A3 || !p->WQ || !p->WK || !p->WV) return RA_ERR_INVALID_ARG;
+  if (p->d != 64 && p->d != 128) return RA_ERR_UNSUPPORTED;
+  // grid limits: B*H blocks in y, and sizes held in 32-bit ints inside the kernels
+  if ((int64_t)p->B * p->H > 65535) return RA_ERR_UNSUPPORTED;
+  if ((int64_t)p->n > (1 << 24)) return RA_ERR_UNSUPPORTED;
+  const void* ptrs[] = {p->A1, p->A2, p->A3, p->WQ, p->WK, p->WV, p->E};
+  for (const void* q : ptrs)
+    if (q && !is_aligned(q, 16)) return RA_ERR_ALIGNMENT;
+  if (p->pos && !is_aligned(p->pos, 4)) return RA_ERR_ALIGNMENT;
+  return RA_OK;
+}
+
+Layout make_layout(const ra_problem* p) {
+  Layout L{};
+  const size_t B = p->B, H = p->H, n = p->n, d = p->d;
+  L.inter = 4;
+  const size_t act = B * H * n * d;
+  const long rows = (long)B * n;
+  long ns = (4 * 148 + 3 * p->H - 1) / (3 * p->H);
+  ns = ns < 1 ? 1 : ns;
+  long maxs = (rows + 63) / 64;
+  if (ns > maxs) ns = maxs;
+  L.nsplit = (int)ns;
+  L.chunk = (int)((rows + ns - 1) / ns);
+  L.nparts = (int)(((n + 31) / 32) * B * H);
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    size_t o = off;
+    off = align_up(off + bytes, kAlignWs);
+    return o;
+  };
+  L.rope = take(n * (d / 2) * sizeof(float2));
+  L.qt = take(act * L.inter);
+  L.kt = take(act * L.inter);
+  L.v = take(act * L.inter);
+  L.ell = take(act * L.inter);
+  L.delta = take(B * H * n * sizeof(float));
+  L.dqt = take(act * sizeof(float));
+  L.dkt = take(act * sizeof(float));
+  L.dv = take(act * sizeof(float));
+  L.dw_part = take(3 * H * (size_t)L.nsplit * d * d * sizeof(float));
+  L.loss_part = take((size_t)L.nparts * sizeof(double));
+  L.total = off;
+  return L;
+}
+
+template <class T>
+T* at(void* ws, size_t off) {
+  return reinterpret_cast<T*>(static_cast<char*>(ws) + off);
+}
+
+ra_status launch_status() {
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? RA_OK : RA_ERR_CUDA;
+}
+
+ra_status check_ws(const ra_problem* p, void* ws, size_t ws_bytes) {
+  if (!ws) return RA_ERR_WORKSPACE;
+  if (!is_aligned(ws, kAlignWs)) return RA_ERR_ALIGNMENT;
+  if (ws_bytes < make_layout(p).total) return RA_ERR_WORKSPACE;
+  return RA_OK;
+}
+
+// ---------------------------------------------------------------------------------------
+// fp32 CUDA-core path
+// ---------------------------------------------------------------------------------------
+template <class T>
+ra_status simt_project(const ra_problem* p, const Layout& L, void* ws, cudaStream_t st) {
+  using namespace ra::simt;
+  const int n = p->n, d = p->d, half = d / 2;
+  float2* tab = at<float2>(ws, L.rope);
+  {
+    int total = n * half;
+    Launch l(K_ROPE_TABLE, st);
+    rope_table_kernel<<<(total + 255) / 256, 256, 0, st>>>(tab, p->pos, n, half, p->rope_base);
+  }
+  {
+    size_t smem = (size_t)(kRows * (d + 4) + d * d) * sizeof(float);
+    auto k = proj_rope_kernel<T, float>;
+    cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    dim3 grid((n + kRows - 1) / kRows, p->B * p->H, 3);
+    Launch l(K_PROJ_SIMT, st);
+    k<<<grid, kThreads, smem, st>>>(
+        (const T*)p->A1, (const T*)p->A2, (const T*)p->A3, (const T*)p->WQ, (const T*)p->WK,
+        (const T*)p->WV, tab, at<float>(ws, L.qt), at<float>(ws, L.kt), at<float>(ws, L.v),
+        p->H, n, d);
+  }
+  return launch_status();
+}
+
+template <class T>
+ra_status simt_fwd(const ra_problem* p, void* O, float* lse, float* loss, void* ws,
+                   cudaStream_t st) {
+  using namespace ra::simt;
+  const Layout L = make_layout(p);
+  ra_status s = simt_project<T>(p, L, ws, st);
+  if (s != RA_OK) return s;
+  const int n = p->n, d = p->d;
+  const float scale = 1.0f / sqrtf((float)d);
+  size_t smem = (size_t)(3 * kRows * (d + 4) + kRows * 33) * sizeof(float);
+  auto k = attn_fwd_kernel<T, T>;
+  cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  dim3 grid((n + kRows - 1) / kRows, p->B * p->H);
+  {
+    Launch l(K_FWD_SIMT, st);
+    k<<<grid, kThreads, smem, st>>>(at<float>(ws, L.qt), at<float>(ws, L.kt), at<float>(ws, L.v),
+                                    (const T*)p->E, (T*)O, lse, at<float>(ws, L.ell),
+                                    at<float>(ws, L.delta), at<double>(ws, L.loss_part), n, d,
+                                    p->causal, scale * ra::kLog2e);
+  }
+  if (loss) {
+    Launch l(K_LOSS, st);
+    loss_finalize_kernel<<<1, 256, 0, st>>>(at<double>(ws, L.loss_part), L.nparts, loss);
+  }
+  return launch_status();
+}
+
+template <class T>
+ra_status simt_bwd(const ra_problem* p, const void* O, const float* lse, float* loss,
+                   float* dWQ, float* dWK, float* dWV, void* ws, int holds, cudaStream_t st) {
+  using namespace ra::simt;
+  const Layout L = make_layout(p);
+  const int n = p->n, d = p->d;
+  if (!holds) {
+    ra_status s = simt_project<T>(p, L, ws, st);
+    if (s != RA_OK) return s;
+    dim3 grid((n + kRows - 1) / kRows, p->B * p->H);
+    Launch l(K_BWD_PRE, st);
+    bwd_pre_kernel<T, float><<<grid, kThreads, 0, st>>>(
+        (const T*)O, (const T*)p->E, at<float>(ws, L.ell), at<float>(ws, L.delta),
+        at<double>(ws, L.loss_part), n, d);
+  }
+  const size_t act = (size_t)p->B * p->H * n * d;
+  if (cudaMemsetAsync(at<float>(ws, L.dqt), 0, act * sizeof(float), st) != cudaSuccess)
+    return RA_ERR_CUDA;
+  const float scale = 1.0f / sqrtf((float)d);
+  {
+    size_t smem = (size_t)(4 * kRows * (d + 4) + 2 * kRows * 33 + 2 * kRows) * sizeof(float);
+    cudaFuncSetAttribute(attn_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)smem);
+    dim3 grid((n + kRows - 1) / kRows, p->B * p->H);
+    Launch l(K_BWD_SIMT, st);
+    attn_bwd_kernel<<<grid, kThreads, smem, st>>>(
+        at<float>(ws, L.qt), at<float>(ws, L.kt), at<float>(ws, L.v), at<float>(ws, L.ell), lse,
+        at<float>(ws, L.delta), at<float>(ws, L.dqt), at<float>(ws, L.dkt), at<float>(ws, L.dv),
+        n, d, p->causal, scale, scale * ra::kLog2e);
+  }
+  {
+    size_t smem = (size_t)2 * 16 * d * sizeof(float);
+    dim3 grid(L.nsplit, 3, p->H);
+    {
+      Launch l(K_DW_PART_SIMT, st);
+      dw_partial_kernel<T, float><<<grid, kThreads, smem, st>>>(
+          (const T*)p->A1, (const T*)p->A2, (const T*)p->A3, at<float>(ws, L.dqt),
+          at<float>(ws, L.dkt), at<float>(ws, L.dv), at<float2>(ws, L.rope),
+          at<float>(ws, L.dw_part), p->B, p->H, n, d, L.chunk);
+    }
+    size_t total = (size_t)3 * p->H * d * d;
+    Launch l(K_DW_REDUCE, st);
+    dw_reduce_kernel<<<(unsigned)((total + 255) / 256), 256, 0, st>>>(
+        at<float>(ws, L.dw_part), dWQ, dWK, dWV, p->H, d, L.nsplit);
+  }
+  if (loss) {
+    Launch l(K_LOSS, st);
+    loss_finalize_kernel<<<1, 256, 0, st>>>(at<double>(ws, L.loss_part), L.nparts, loss);
+  }
+  return launch_status();
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t rope_attn_workspace_bytes(const ra_problem* p) {
+  if (check_problem(p) != RA_OK) return 0;
+  return make_layout(p).total;
+}
+
+ra_status rope_attn_fwd(const ra_problem* p, void* O, float* lse, float* loss, void* ws,
+                        size_t ws_bytes, void* stream) {
+  ra_status s = check_problem(p);
+  if (s != RA_OK) return s;
+  if (!O || !lse) return RA_ERR_INVALID_ARG;
+  if (loss && !p->E) return RA_ERR_INVALID_ARG;
+  if (!is_aligned(O, 16) || !is_aligned(lse, 4) || (loss && !is_aligned(loss, 4)))
+    return RA_ERR_ALIGNMENT;
+  s = check_ws(p, ws, ws_bytes);
+  if (s != RA_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (p->dtype == RA_F32) return simt_fwd<float>(p, O, lse, loss, ws, st);
+  return simt_fwd<__nv_bfloat16>(p, O, lse, loss, ws, st);
+}
+
+ra_status rope_attn_loss_bwd(const ra_problem* p, const void* O, const float* lse, float* loss,
+                             float* dWQ, float* dWK, float* dWV, void* ws, size_t ws_bytes,
+                             int32_t ws_holds_fwd, void* stream) {
+  ra_status s = check_problem(p);
+  if (s != RA_OK) return s;
+  if (!p->E || !O || !lse || !dWQ || !dWK || !dWV) return RA_ERR_INVALID_ARG;
+  if (ws_holds_fwd != 0 && ws_holds_fwd != 1) return RA_ERR_INVALID_ARG;
+  if (!is_aligned(O, 16) || !is_aligned(lse, 4) || (loss && !is_aligned(loss, 4)) ||
+      !is_aligned(dWQ, 16) || !is_aligned(dWK, 16) || !is_aligned(dWV, 16))
+    return RA_ERR_ALIGNMENT;
+  s = check_ws(p, ws, ws_bytes);
+  if (s != RA_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (p->dtype == RA_F32)
+    return simt_bwd<float>(p, O, lse, loss, dWQ, dWK, dWV, ws, ws_holds_fwd, st);
+  return simt_bwd<__nv_bfloat16>(p, O, lse, loss, dWQ, dWK, dWV, ws, ws_holds_fwd, st);
+}
+
+ra_status rope_attn_last_error(void* stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return RA_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, ra::g_status, sizeof(int)) != cudaSuccess) return RA_ERR_CUDA;
+  if (v != 0) {
+    int zero = 0;
+    if (cudaMemcpyToSymbol(ra::g_status, &zero, sizeof(int)) != cudaSuccess) return RA_ERR_CUDA;
+    return RA_ERR_TIMEOUT;
+  }
+  return RA_OK;
+}
+
+const char* rope_attn_status_string(ra_status s) {
+  switch (s) {
+    case RA_OK: return "RA_OK";
+    case RA_ERR_INVALID_ARG: return "RA_ERR_INVALID_ARG: null pointer, bad size or flag";
+    case RA_ERR_UNSUPPORTED: return "RA_ERR_UNSUPPORTED: head dimension or size not supported";
+    case RA_ERR_ALIGNMENT: return "RA_ERR_ALIGNMENT: device pointer not aligned";
+    case RA_ERR_WORKSPACE: return "RA_ERR_WORKSPACE: workspace missing or too small";
+    case RA_ERR_CUDA: return "RA_ERR_CUDA: CUDA launch or runtime call failed";
+    case RA_ERR_TIMEOUT: return "RA_ERR_TIMEOUT: a kernel gave up waiting on a barrier";
+  }
+  return "unknown ra_status";
+}
+
+int64_t rope_attn_launch_count(void) {
+  int64_t v = t_launches;
+  t_launches = 0;
+  return v;
+}
+
+void rope_attn_profile_enable(int32_t on) {
+  t_prof.on = on != 0;
+  if (!t_prof.on) t_prof.recycle();
+}
+
+int32_t rope_attn_profile_read(float* ms, int32_t* launches, int32_t max_kernels) {
+  for (int k = 0; k < max_kernels && k < K_COUNT; ++k) {
+    if (ms) ms[k] = 0.f;
+    if (launches) launches[k] = 0;
+  }
+  int32_t ret = K_COUNT;
+  for (auto& r : t_prof.recs) {
+    float t = 0.f;
+    if (cudaEventSynchronize(r.stop) != cudaSuccess ||
+        cudaEventElapsedTime(&t, r.start, r.stop) != cudaSuccess) {
+      ret = -1;
+      continue;
+    }
+    if (r.id < max_kernels) {
+      if (ms) ms[r.id] += t;
+      if (launches) launches[r.id] += 1;
+    }
+  }
+  t_prof.recycle();
+  return ret;
+}
+
+const char* rope_attn_kernel_name(int32_t id) {
+  return (id >= 0 && id < K_COUNT) ? kKernelNames[id] : nullptr;
+}
+
+}  // extern "C"

@@ -1,0 +1,452 @@
+// fp32 CUDA-core kernels: the precision path for fp32 I/O.  Same math as the tensor-core
+// path, all products and sums in fp32; intermediate Q~, K~, V, l kept in fp32.
+//
+// Definitions followed ("RoPE Attention kan bijna lineair worden getraind", Methodologie 1
+// and 2): s = softmax of the scaled scores, l = O - E, beta = l V^T,
+// gamma = diag(s) beta - s s^T beta evaluated row-wise as s_i o (beta_i - <l_i, O_i>).
+#pragma once
+#include "common.cuh"
+
+namespace ra {
+namespace simt {
+
+constexpr int kRows = 32;      // query (or key) rows per block
+constexpr int kThreads = 256;  // 8 threads per row
+
+// ---------------------------------------------------------------------------------------
+// RoPE table: tab[i][k] = (cos, sin)(pos_i * base^(-2k/d)), angle and sin/cos in fp64.
+// ---------------------------------------------------------------------------------------
+__global__ void rope_table_kernel(float2* __restrict__ tab, const int32_t* __restrict__ pos,
+                                  int n, int half, double base) {
+  int idx = blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= n * half) return;
+  int i = idx / half, k = idx - i * half;
+  double p = pos ? (double)pos[i] : (double)i;
+  double theta = pow(base, -2.0 * (double)k / (double)(2 * half));
+  double s, c;
+  sincos(p * theta, &s, &c);
+  tab[idx] = make_float2((float)c, (float)s);
+}
+
+// ---------------------------------------------------------------------------------------
+// Projection + RoPE: out_z = rot(A_z W_z) for z = 0 (Q), 1 (K); out_2 = A3 WV (no rotation).
+// grid (ceil(n/32), B*H, 3), 256 threads, dynamic smem (32*(d+4) + d*d) floats.
+// ---------------------------------------------------------------------------------------
+template <class TI, class TO>
+__global__ void __launch_bounds__(kThreads)
+proj_rope_kernel(const TI* __restrict__ A1, const TI* __restrict__ A2, const TI* __restrict__ A3,
+                 const TI* __restrict__ WQ, const TI* __restrict__ WK, const TI* __restrict__ WV,
+                 const float2* __restrict__ tab, TO* __restrict__ Qt, TO* __restrict__ Kt,
+                 TO* __restrict__ Vo, int H, int n, int d) {
+  extern __shared__ float smem[];
+  const int ld = d + 4;
+  float* As = smem;             // [32][d+4]
+  float* Ws = smem + kRows * ld;  // [d][d]
+  const int z = blockIdx.z, bh = blockIdx.y, h = bh % H;
+  const int i0 = blockIdx.x * kRows;
+  const TI* A = (z == 0 ? A1 : z == 1 ? A2 : A3) + ((size_t)bh * n + i0) * d;
+  const TI* W = (z == 0 ? WQ : z == 1 ? WK : WV) + (size_t)h * d * d;
+  TO* out = (z == 0 ? Qt : z == 1 ? Kt : Vo) + ((size_t)bh * n + i0) * d;
+  const int tid = threadIdx.x;
+  load_tile_f32(As, ld, A, kRows, d, min(kRows, n - i0), tid, kThreads);
+  for (int e = tid; e < d * d; e += kThreads) Ws[e] = to_f(W[e]);
+  __syncthreads();
+  const int r = tid >> 3, g = tid & 7;
+  const int row = i0 + r;
+  const int half = d >> 1;
+  for (int pk = g; pk < half; pk += 8) {
+    float a0 = 0.f, a1 = 0.f;
+    for (int i = 0; i < d; ++i) {
+      float a = As[r * ld + i];
+      float2 w = *reinterpret_cast<const float2*>(&Ws[i * d + 2 * pk]);
+      a0 = fmaf(a, w.x, a0);
+      a1 = fmaf(a, w.y, a1);
+    }
+    if (row < n) {
+      float o0 = a0, o1 = a1;
+      if (z < 2) {
+        float2 cs = tab[(size_t)row * half + pk];
+        o0 = a0 * cs.x - a1 * cs.y;
+        o1 = a0 * cs.y + a1 * cs.x;
+      }
+      out[(size_t)r * d + 2 * pk] = from_f<TO>(o0);
+      out[(size_t)r * d + 2 * pk + 1] = from_f<TO>(o1);
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------------------
+// Forward: online softmax over key tiles of 32, O = s V, LSE; with a target E also
+// l = O - E, delta_i = <l_i, O_i> and per-block partial sums of 1/2 l^2.
+// grid (ceil(n/32), B*H), 256 threads; thread (r = tid/8, g = tid%8).
+// ---------------------------------------------------------------------------------------
+template <class TE, class TO>
+__global__ void __launch_bounds__(kThreads)
+attn_fwd_kernel(const float* __restrict__ Qt, const float* __restrict__ Kt,
+                const float* __restrict__ V, const TE* __restrict__ E, TO* __restrict__ O,
+                float* __restrict__ lse, float* __restrict__ ell, float* __restrict__ delta,
+                double* __restrict__ loss_part, int n, int d, int causal, float scale_log2) {
+  extern __shared__ float smem[];
+  const int ld = d + 4;
+  float* Qs = smem;
+  float* Ks = Qs + kRows * ld;
+  float* Vs = Ks + kRows * ld;
+  float* Ps = Vs + kRows * ld;  // [32][33]
+  __shared__ double red[kThreads / 32];
+  const int bh = blockIdx.y, i0 = blockIdx.x * kRows, tid = threadIdx.x;
+  const int r = tid >> 3, g = tid & 7;
+  const int row = i0 + r;
+  const size_t base = (size_t)bh * n * d;
+  load_tile_f32(Qs, ld, Qt + base + (size_t)i0 * d, kRows, d, min(kRows, n - i0), tid, kThreads);
+  float acc[16];
+  const int ncol = d >> 3;  // columns g + 8u per thread
+#pragma unroll
+  for (int u = 0; u < 16; ++u) acc[u] = 0.f;
+  float m = -INFINITY, l = 0.f;
+  const int jend = causal ? min(n, i0 + kRows) : n;
+  for (int j0 = 0; j0 < jend; j0 += kRows) {
+    __syncthreads();
+    load_tile_f32(Ks, ld, Kt + base + (size_t)j0 * d, kRows, d, min(kRows, n - j0), tid, kThreads);
+    load_tile_f32(Vs, ld, V + base + (size_t)j0 * d, kRows, d, min(kRows, n - j0), tid, kThreads);
+    __syncthreads();
+    float s[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) s[q] = 0.f;
+    for (int c = 0; c < d; c += 4) {
+      float4 qv = *reinterpret_cast<const float4*>(&Qs[r * ld + c]);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        float4 kv = *reinterpret_cast<const float4*>(&Ks[(g + 8 * q) * ld + c]);
+        s[q] = fmaf(qv.x, kv.x, fmaf(qv.y, kv.y, fmaf(qv.z, kv.z, fmaf(qv.w, kv.w, s[q]))));
+      }
+    }
+    float tmax = -INFINITY;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      int key = j0 + g + 8 * q;
+      bool ok = key < n && (!causal || key <= row);
+      s[q] = ok ? s[q] * scale_log2 : -INFINITY;
+      tmax = fmaxf(tmax, s[q]);
+    }
+#pragma unroll
+    for (int o = 1; o < 8; o <<= 1) tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, o));
+    const float mnew = fmaxf(m, tmax);
+    const float mref = (mnew == -INFINITY) ? 0.f : mnew;
+    const float alpha = exp2f(m - mref);
+    float psum = 0.f;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      float p = exp2f(s[q] - mref);
+      psum += p;
+      Ps[r * 33 + g + 8 * q] = p;
+    }
+#pragma unroll
+    for (int o = 1; o < 8; o <<= 1) psum += __shfl_xor_sync(0xffffffffu, psum, o);
+    l = l * alpha + psum;
+    m = mnew;
+    __syncthreads();
+#pragma unroll
+    for (int u = 0; u < 16; ++u) acc[u] *= alpha;
+    for (int k = 0; k < kRows; ++k) {
+      float p = Ps[r * 33 + k];
+#pragma unroll
+      for (int u = 0; u < 16; ++u)
+        if (u < ncol) acc[u] = fmaf(p, Vs[k * ld + g + 8 * u], acc[u]);
+    }
+  }
+  const float inv = 1.f / l;
+  const bool vrow = row < n;
+  const size_t ro = base + (size_t)row * d;
+  float dl = 0.f, sq = 0.f;
+#pragma unroll
+  for (int u = 0; u < 16; ++u) {
+    if (u < ncol && vrow) {
+      const int col = g + 8 * u;
+      const float o = acc[u] * inv;
+      O[ro + col] = from_f<TO>(o);
+      if (E) {
+        const float e = o - to_f(E[ro + col]);
+        ell[ro + col] = e;
+        dl = fmaf(e, o, dl);
+        sq = fmaf(e, e, sq);
+      }
+    }
+  }
+#pragma unroll
+  for (int o = 1; o < 8; o <<= 1) {
+    dl += __shfl_xor_sync(0xffffffffu, dl, o);
+    sq += __shfl_xor_sync(0xffffffffu, sq, o);
+  }
+  if (vrow && g == 0) {
+    lse[(size_t)bh * n + row] = (m + log2f(l)) * kLn2;
+    if (E) delta[(size_t)bh * n + row] = dl;
+  }
+  double part = (vrow && g == 0) ? 0.5 * (double)sq : 0.0;
+  if (E) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+    if ((tid & 31) == 0) red[tid >> 5] = part;
+    __syncthreads();
+    if (tid == 0) {
+      double t = 0.0;
+      for (int w = 0; w < kThreads / 32; ++w) t += red[w];
+      loss_part[(size_t)blockIdx.y * gridDim.x + blockIdx.x] = t;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------------------
+// l = O - E, delta_i = <l_i, O_i>, partial sums of 1/2 l^2, from a given O (I/O dtype).
+// grid (ceil(n/32), B*H), 256 threads.
+// ---------------------------------------------------------------------------------------
+template <class T, class TL>
+__global__ void __launch_bounds__(kThreads)
+bwd_pre_kernel(const T* __restrict__ O, const T* __restrict__ E, TL* __restrict__ ell,
+               float* __restrict__ delta, double* __restrict__ loss_part, int n, int d) {
+  __shared__ double red[kThreads / 32];
+  const int bh = blockIdx.y, tid = threadIdx.x, r = tid >> 3, g = tid & 7;
+  const int row = blockIdx.x * kRows + r;
+  float dl = 0.f, sq = 0.f;
+  if (row < n) {
+    const size_t ro = ((size_t)bh * n + row) * d;
+    for (int col = g; col < d; col += 8) {
+      float o = to_f(O[ro + col]);
+      float e = o - to_f(E[ro + col]);
+      ell[ro + col] = from_f<TL>(e);
+      dl = fmaf(e, o, dl);
+      sq = fmaf(e, e, sq);
+    }
+  }
+#pragma unroll
+  for (int o = 1; o < 8; o <<= 1) {
+    dl += __shfl_xor_sync(0xffffffffu, dl, o);
+    sq += __shfl_xor_sync(0xffffffffu, sq, o);
+  }
+  if (row < n && g == 0) delta[(size_t)bh * n + row] = dl;
+  double part = (row < n && g == 0) ? 0.5 * (double)sq : 0.0;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+  if ((tid & 31) == 0) red[tid >> 5] = part;
+  __syncthreads();
+  if (tid == 0) {
+    double t = 0.0;
+    for (int w = 0; w < kThreads / 32; ++w) t += red[w];
+    loss_part[(size_t)blockIdx.y * gridDim.x + blockIdx.x] = t;
+  }
+}
+
+// ---------------------------------------------------------------------------------------
+// Backward over one key tile of 32 rows, looping over query tiles of 32:
+//   P^T = exp(S^T - lse), beta^T = V l^T, gamma^T = P^T o (beta^T - delta)
+//   dV += P^T l,  dK~ += gamma^T Q~ / sqrt(d),  dQ~ += gamma K~ / sqrt(d) (atomic adds)
+// grid (ceil(n/32), B*H), 256 threads, thread (r = tid/8, g = tid%8).
+// ---------------------------------------------------------------------------------------
+__global__ void __launch_bounds__(kThreads)
+attn_bwd_kernel(const float* __restrict__ Qt, const float* __restrict__ Kt,
+                const float* __restrict__ V, const float* __restrict__ ell,
+                const float* __restrict__ lse, const float* __restrict__ delta,
+                float* __restrict__ dQt, float* __restrict__ dKt, float* __restrict__ dV,
+                int n, int d, int causal, float scale, float scale_log2) {
+  extern __shared__ float smem[];
+  const int ld = d + 4;
+  float* Ks = smem;
+  float* Vs = Ks + kRows * ld;
+  float* Qs = Vs + kRows * ld;
+  float* Ls = Qs + kRows * ld;
+  float* PT = Ls + kRows * ld;   // [32][33]
+  float* GT = PT + kRows * 33;   // [32][33]
+  float* lse_s = GT + kRows * 33;
+  float* del_s = lse_s + kRows;
+  const int bh = blockIdx.y, j0 = blockIdx.x * kRows, tid = threadIdx.x;
+  const int r = tid >> 3, g = tid & 7;
+  const int key = j0 + r;
+  const size_t base = (size_t)bh * n * d;
+  const int ncol = d >> 3;
+  load_tile_f32(Ks, ld, Kt + base + (size_t)j0 * d, kRows, d, min(kRows, n - j0), tid, kThreads);
+  load_tile_f32(Vs, ld, V + base + (size_t)j0 * d, kRows, d, min(kRows, n - j0), tid, kThreads);
+  float adk[16], adv[16];
+#pragma unroll
+  for (int u = 0; u < 16; ++u) adk[u] = adv[u] = 0.f;
+  const int istart = causal ? j0 : 0;
+  for (int i0 = istart; i0 < n; i0 += kRows) {
+    __syncthreads();
+    const int vr = min(kRows, n - i0);
+    load_tile_f32(Qs, ld, Qt + base + (size_t)i0 * d, kRows, d, vr, tid, kThreads);
+    load_tile_f32(Ls, ld, ell + base + (size_t)i0 * d, kRows, d, vr, tid, kThreads);
+    if (tid < kRows) {
+      lse_s[tid] = (tid < vr) ? lse[(size_t)bh * n + i0 + tid] * kLog2e : 0.f;
+      del_s[tid] = (tid < vr) ? delta[(size_t)bh * n + i0 + tid] : 0.f;
+    }
+    __syncthreads();
+    float s[4], b[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) s[q] = b[q] = 0.f;
+    for (int c = 0; c < d; c += 4) {
+      float4 kv = *reinterpret_cast<const float4*>(&Ks[r * ld + c]);
+      float4 vv = *reinterpret_cast<const float4*>(&Vs[r * ld + c]);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        float4 qv = *reinterpret_cast<const float4*>(&Qs[(g + 8 * q) * ld + c]);
+        float4 lv = *reinterpret_cast<const float4*>(&Ls[(g + 8 * q) * ld + c]);
+        s[q] = fmaf(kv.x, qv.x, fmaf(kv.y, qv.y, fmaf(kv.z, qv.z, fmaf(kv.w, qv.w, s[q]))));
+        b[q] = fmaf(vv.x, lv.x, fmaf(vv.y, lv.y, fmaf(vv.z, lv.z, fmaf(vv.w, lv.w, b[q]))));
+      }
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int qi = g + 8 * q, qrow = i0 + qi;
+      const bool ok = key < n && qrow < n && (!causal || key <= qrow);
+      const float p = ok ? exp2f(s[q] * scale_log2 - lse_s[qi]) : 0.f;
+      PT[r * 33 + qi] = p;
+      GT[r * 33 + qi] = p * (b[q] - del_s[qi]);
+    }
+    __syncthreads();
+    for (int k = 0; k < kRows; ++k) {
+      const float p = PT[r * 33 + k], gm = GT[r * 33 + k];
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        if (u < ncol) {
+          adv[u] = fmaf(p, Ls[k * ld + g + 8 * u], adv[u]);
+          adk[u] = fmaf(gm, Qs[k * ld + g + 8 * u], adk[u]);
+        }
+      }
+    }
+    // dQ~ rows of this query tile: thread (r -> query row, g -> columns)
+    const int qrow = i0 + r;
+    if (qrow < n) {
+      float aq[16];
+#pragma unroll
+      for (int u = 0; u < 16; ++u) aq[u] = 0.f;
+      for (int k = 0; k < kRows; ++k) {
+        const float gm = GT[k * 33 + r];
+#pragma unroll
+        for (int u = 0; u < 16; ++u)
+          if (u < ncol) aq[u] = fmaf(gm, Ks[k * ld + g + 8 * u], aq[u]);
+      }
+      float* dst = dQt + base + (size_t)qrow * d;
+#pragma unroll
+      for (int u = 0; u < 16; ++u)
+        if (u < ncol) atomicAdd(dst + g + 8 * u, aq[u] * scale);
+    }
+  }
+  if (key < n) {
+    const size_t ro = base + (size_t)key * d;
+#pragma unroll
+    for (int u = 0; u < 16; ++u) {
+      if (u < ncol) {
+        dKt[ro + g + 8 * u] = adk[u] * scale;
+        dV[ro + g + 8 * u] = adv[u];
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------------------
+// Weight-gradient partial sums over a chunk of the B*n rows of one head:
+//   part[z][h][split] = sum_rows A_z[row]^T dX_z[row], dX_0 = rot^-1(dQ~), dX_1 = rot^-1(dK~),
+//   dX_2 = dV.  grid (nsplit, 3, H), 256 threads, each an (d/16) x (d/16) sub-tile.
+// ---------------------------------------------------------------------------------------
+template <class TA, class TX>
+__global__ void __launch_bounds__(kThreads)
+dw_partial_kernel(const TA* __restrict__ A1, const TA* __restrict__ A2, const TA* __restrict__ A3,
+                  const TX* __restrict__ dQt, const TX* __restrict__ dKt, const TX* __restrict__ dV,
+                  const float2* __restrict__ tab, float* __restrict__ part, int B, int H, int n,
+                  int d, int chunk) {
+  constexpr int kR = 16;
+  extern __shared__ float smem[];
+  float* As = smem;            // [16][d]
+  float* Xs = smem + kR * d;   // [16][d]
+  const int split = blockIdx.x, z = blockIdx.y, h = blockIdx.z, nsplit = gridDim.x;
+  const TA* A = z == 0 ? A1 : z == 1 ? A2 : A3;
+  const TX* X = z == 0 ? dQt : z == 1 ? dKt : dV;
+  const int tid = threadIdx.x, sub = d >> 4;
+  const int ti = (tid >> 4) * sub, tj = (tid & 15) * sub;
+  float acc[8][8];
+#pragma unroll
+  for (int a = 0; a < 8; ++a)
+#pragma unroll
+    for (int c = 0; c < 8; ++c) acc[a][c] = 0.f;
+  const long total = (long)B * n;
+  const long r0 = (long)split * chunk, r1 = min(total, r0 + chunk);
+  const int half = d >> 1;
+  for (long rb = r0; rb < r1; rb += kR) {
+    __syncthreads();
+    for (int e = tid; e < kR * half; e += kThreads) {
+      const int rr = e / half, pk = e - rr * half;
+      const long gr = rb + rr;
+      float a0 = 0.f, a1 = 0.f, x0 = 0.f, x1 = 0.f;
+      if (gr < r1) {
+        const int b = (int)(gr / n), i = (int)(gr - (long)b * n);
+        const size_t off = (((size_t)b * H + h) * n + i) * d + 2 * pk;
+        a0 = to_f(A[off]);
+        a1 = to_f(A[off + 1]);
+        float y0 = to_f(X[off]), y1 = to_f(X[off + 1]);
+        if (z < 2) {
+          // inverse rotation: angle -phi
+          float2 cs = tab[(size_t)i * half + pk];
+          x0 = y0 * cs.x + y1 * cs.y;
+          x1 = -y0 * cs.y + y1 * cs.x;
+        } else {
+          x0 = y0;
+          x1 = y1;
+        }
+      }
+      As[rr * d + 2 * pk] = a0;
+      As[rr * d + 2 * pk + 1] = a1;
+      Xs[rr * d + 2 * pk] = x0;
+      Xs[rr * d + 2 * pk + 1] = x1;
+    }
+    __syncthreads();
+    for (int k = 0; k < kR; ++k) {
+      float av[8], xv[8];
+#pragma unroll
+      for (int a = 0; a < 8; ++a) {
+        av[a] = a < sub ? As[k * d + ti + a] : 0.f;
+        xv[a] = a < sub ? Xs[k * d + tj + a] : 0.f;
+      }
+#pragma unroll
+      for (int a = 0; a < 8; ++a)
+#pragma unroll
+        for (int c = 0; c < 8; ++c) acc[a][c] = fmaf(av[a], xv[c], acc[a][c]);
+    }
+  }
+  float* dst = part + (((size_t)z * H + h) * nsplit + split) * d * d;
+  for (int a = 0; a < sub; ++a)
+    for (int c = 0; c < sub; ++c) dst[(size_t)(ti + a) * d + tj + c] = acc[a][c];
+}
+
+// dW[z][h] = sum over splits (fixed order) of part[z][h][split].
+__global__ void dw_reduce_kernel(const float* __restrict__ part, float* __restrict__ dWQ,
+                                 float* __restrict__ dWK, float* __restrict__ dWV, int H, int d,
+                                 int nsplit) {
+  const size_t dd = (size_t)d * d;
+  const size_t idx = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= 3 * H * dd) return;
+  const int z = (int)(idx / (H * dd));
+  const size_t rem = idx - (size_t)z * H * dd;
+  const int h = (int)(rem / dd);
+  const size_t e = rem - (size_t)h * dd;
+  const float* src = part + ((size_t)z * H + h) * nsplit * dd + e;
+  double s = 0.0;
+  for (int k = 0; k < nsplit; ++k) s += (double)src[(size_t)k * dd];
+  float* dW = z == 0 ? dWQ : z == 1 ? dWK : dWV;
+  dW[(size_t)h * dd + e] = (float)s;
+}
+
+// loss = sum of the partials in a fixed order (fp64), one block of 256 threads.
+__global__ void loss_finalize_kernel(const double* __restrict__ part, int count,
+                                     float* __restrict__ loss) {
+  __shared__ double red[256];
+  double s = 0.0;
+  for (int i = threadIdx.x; i < count; i += blockDim.x) s += part[i];
+  red[threadIdx.x] = s;
+  __syncthreads();
+  for (int w = blockDim.x / 2; w > 0; w >>= 1) {
+    if ((int)threadIdx.x < w) red[threadIdx.x] += red[threadIdx.x + w];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) *loss = (float)red[0];
+}
+
+}  // namespace simt
+}  // namespace ra
