@@ -10,9 +10,13 @@
 
 #include <vector>
 
+#include <cudaTypedefs.h>
+#include <stdlib.h>
+
 #include "../../include/rope_attn.h"
 #include "common.cuh"
 #include "simt_kernels.cuh"
+#include "tc_attn_fwd.cuh"
 
 namespace {
 
@@ -28,11 +32,13 @@ enum KernelId : int {
   K_DW_PART_SIMT,
   K_DW_REDUCE,
   K_LOSS,
+  K_FWD_TC,
   K_COUNT
 };
 const char* const kKernelNames[K_COUNT] = {
     "rope_table", "proj_rope_simt", "attn_fwd_simt", "bwd_pre",
-    "attn_bwd_simt", "dw_partial_simt", "dw_reduce", "loss_finalize"};
+    "attn_bwd_simt", "dw_partial_simt", "dw_reduce", "loss_finalize",
+    "attn_fwd_tc"};
 
 struct ProfRecord {
   int id;
@@ -99,7 +105,9 @@ struct Layout {
   int inter;         // bytes per intermediate element
   int nsplit;        // weight-gradient row splits per head
   int chunk;         // rows per split
-  int nparts;        // loss partial sums
+  int nparts;        // capacity of the loss partial sums
+  int nparts_fwd;    // partial sums the forward writes
+  int nparts_pre;    // partial sums the backward's own l = O - E pass writes
 };
 
 bool is_aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
@@ -125,7 +133,7 @@ ra_status check_problem(const ra_problem* p) {
 Layout make_layout(const ra_problem* p) {
   Layout L{};
   const size_t B = p->B, H = p->H, n = p->n, d = p->d;
-  L.inter = 4;
+  L.inter = p->dtype == RA_BF16 ? 2 : 4;
   const size_t act = B * H * n * d;
   const long rows = (long)B * n;
   long ns = (4 * 148 + 3 * p->H - 1) / (3 * p->H);
@@ -134,7 +142,9 @@ Layout make_layout(const ra_problem* p) {
   if (ns > maxs) ns = maxs;
   L.nsplit = (int)ns;
   L.chunk = (int)((rows + ns - 1) / ns);
-  L.nparts = (int)(((n + 31) / 32) * B * H);
+  L.nparts_pre = (int)(((n + 31) / 32) * B * H);
+  L.nparts_fwd = p->dtype == RA_BF16 ? (int)(((n + 127) / 128) * B * H) : L.nparts_pre;
+  L.nparts = L.nparts_pre;
   size_t off = 0;
   auto take = [&](size_t bytes) {
     size_t o = off;
@@ -173,10 +183,55 @@ ra_status check_ws(const ra_problem* p, void* ws, size_t ws_bytes) {
   return RA_OK;
 }
 
+// Bound on every on-chip wait inside the tensor-core kernels (RA_WAIT_LIMIT_MS, default 2 s).
+unsigned long long wait_limit_ns() {
+  static unsigned long long v = [] {
+    const char* e = getenv("RA_WAIT_LIMIT_MS");
+    long ms = e ? atol(e) : 2000;
+    if (ms <= 0) ms = 2000;
+    return (unsigned long long)ms * 1000000ull;
+  }();
+  return v;
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return (EncodeTiledFn) nullptr;
+    return reinterpret_cast<EncodeTiledFn>(f);
+  }();
+  return fn;
+}
+
+// 3-D map over bf16 rows [outer][rows][cols] with a box of 64 columns x box_rows rows and
+// 128-byte swizzle; rows past `rows` of each outer index read as zero.
+bool map_bf16_3d(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows,
+                 uint64_t outer, uint32_t box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {cols, rows, outer};
+  cuuint64_t strides[2] = {cols * 2, rows * cols * 2};
+  cuuint32_t box[3] = {64, box_rows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
 // ---------------------------------------------------------------------------------------
 // fp32 CUDA-core path
 // ---------------------------------------------------------------------------------------
-template <class T>
+template <class T, class TX>
 ra_status simt_project(const ra_problem* p, const Layout& L, void* ws, cudaStream_t st) {
   using namespace ra::simt;
   const int n = p->n, d = p->d, half = d / 2;
@@ -188,14 +243,13 @@ ra_status simt_project(const ra_problem* p, const Layout& L, void* ws, cudaStrea
   }
   {
     size_t smem = (size_t)(kRows * (d + 4) + d * d) * sizeof(float);
-    auto k = proj_rope_kernel<T, float>;
+    auto k = proj_rope_kernel<T, TX>;
     cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     dim3 grid((n + kRows - 1) / kRows, p->B * p->H, 3);
     Launch l(K_PROJ_SIMT, st);
     k<<<grid, kThreads, smem, st>>>(
         (const T*)p->A1, (const T*)p->A2, (const T*)p->A3, (const T*)p->WQ, (const T*)p->WK,
-        (const T*)p->WV, tab, at<float>(ws, L.qt), at<float>(ws, L.kt), at<float>(ws, L.v),
-        p->H, n, d);
+        (const T*)p->WV, tab, at<TX>(ws, L.qt), at<TX>(ws, L.kt), at<TX>(ws, L.v), p->H, n, d);
   }
   return launch_status();
 }
@@ -205,7 +259,7 @@ ra_status simt_fwd(const ra_problem* p, void* O, float* lse, float* loss, void* 
                    cudaStream_t st) {
   using namespace ra::simt;
   const Layout L = make_layout(p);
-  ra_status s = simt_project<T>(p, L, ws, st);
+  ra_status s = simt_project<T, float>(p, L, ws, st);
   if (s != RA_OK) return s;
   const int n = p->n, d = p->d;
   const float scale = 1.0f / sqrtf((float)d);
@@ -222,24 +276,75 @@ ra_status simt_fwd(const ra_problem* p, void* O, float* lse, float* loss, void* 
   }
   if (loss) {
     Launch l(K_LOSS, st);
-    loss_finalize_kernel<<<1, 256, 0, st>>>(at<double>(ws, L.loss_part), L.nparts, loss);
+    loss_finalize_kernel<<<1, 256, 0, st>>>(at<double>(ws, L.loss_part), L.nparts_fwd, loss);
   }
   return launch_status();
 }
 
-template <class T>
+// ---------------------------------------------------------------------------------------
+// bf16 tensor-core path
+// ---------------------------------------------------------------------------------------
+template <int D>
+ra_status tc_fwd_launch(const ra_problem* p, const Layout& L, void* O, float* lse, void* ws,
+                        cudaStream_t st) {
+  using namespace ra::tc;
+  using C = FwdCfg<D>;
+  const int n = p->n, BH = p->B * p->H;
+  CUtensorMap mq, mk, mv;
+  if (!map_bf16_3d(&mq, at<void>(ws, L.qt), D, n, BH, 128) ||
+      !map_bf16_3d(&mk, at<void>(ws, L.kt), D, n, BH, 128) ||
+      !map_bf16_3d(&mv, at<void>(ws, L.v), D, n, BH, 128))
+    return RA_ERR_CUDA;
+  FwdParams fp;
+  fp.E = (const __nv_bfloat16*)p->E;
+  fp.O = (__nv_bfloat16*)O;
+  fp.lse = lse;
+  fp.ell = at<__nv_bfloat16>(ws, L.ell);
+  fp.delta = at<float>(ws, L.delta);
+  fp.loss_part = at<double>(ws, L.loss_part);
+  fp.n = n;
+  fp.BH = BH;
+  fp.nq = (n + C::BM - 1) / C::BM;
+  fp.causal = p->causal;
+  fp.scale_log2 = ra::kLog2e / sqrtf((float)D);
+  fp.limit_ns = wait_limit_ns();
+  auto k = attn_fwd_tc_kernel<D>;
+  cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_ALLOC);
+  dim3 grid(BH, fp.nq);
+  Launch l(K_FWD_TC, st);
+  k<<<grid, C::THREADS, C::SMEM_ALLOC, st>>>(mq, mk, mv, fp);
+  return RA_OK;
+}
+
+ra_status tc_fwd(const ra_problem* p, void* O, float* lse, float* loss, void* ws,
+                 cudaStream_t st) {
+  const Layout L = make_layout(p);
+  ra_status s = simt_project<__nv_bfloat16, __nv_bfloat16>(p, L, ws, st);
+  if (s != RA_OK) return s;
+  s = p->d == 128 ? tc_fwd_launch<128>(p, L, O, lse, ws, st)
+                  : tc_fwd_launch<64>(p, L, O, lse, ws, st);
+  if (s != RA_OK) return s;
+  if (loss) {
+    Launch l(K_LOSS, st);
+    ra::simt::loss_finalize_kernel<<<1, 256, 0, st>>>(at<double>(ws, L.loss_part), L.nparts_fwd,
+                                                      loss);
+  }
+  return launch_status();
+}
+
+template <class T, class TX>
 ra_status simt_bwd(const ra_problem* p, const void* O, const float* lse, float* loss,
                    float* dWQ, float* dWK, float* dWV, void* ws, int holds, cudaStream_t st) {
   using namespace ra::simt;
   const Layout L = make_layout(p);
   const int n = p->n, d = p->d;
   if (!holds) {
-    ra_status s = simt_project<T>(p, L, ws, st);
+    ra_status s = simt_project<T, TX>(p, L, ws, st);
     if (s != RA_OK) return s;
     dim3 grid((n + kRows - 1) / kRows, p->B * p->H);
     Launch l(K_BWD_PRE, st);
-    bwd_pre_kernel<T, float><<<grid, kThreads, 0, st>>>(
-        (const T*)O, (const T*)p->E, at<float>(ws, L.ell), at<float>(ws, L.delta),
+    bwd_pre_kernel<T, TX><<<grid, kThreads, 0, st>>>(
+        (const T*)O, (const T*)p->E, at<TX>(ws, L.ell), at<float>(ws, L.delta),
         at<double>(ws, L.loss_part), n, d);
   }
   const size_t act = (size_t)p->B * p->H * n * d;
@@ -248,12 +353,12 @@ ra_status simt_bwd(const ra_problem* p, const void* O, const float* lse, float* 
   const float scale = 1.0f / sqrtf((float)d);
   {
     size_t smem = (size_t)(4 * kRows * (d + 4) + 2 * kRows * 33 + 2 * kRows) * sizeof(float);
-    cudaFuncSetAttribute(attn_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaFuncSetAttribute(attn_bwd_kernel<TX>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          (int)smem);
     dim3 grid((n + kRows - 1) / kRows, p->B * p->H);
     Launch l(K_BWD_SIMT, st);
-    attn_bwd_kernel<<<grid, kThreads, smem, st>>>(
-        at<float>(ws, L.qt), at<float>(ws, L.kt), at<float>(ws, L.v), at<float>(ws, L.ell), lse,
+    attn_bwd_kernel<TX><<<grid, kThreads, smem, st>>>(
+        at<TX>(ws, L.qt), at<TX>(ws, L.kt), at<TX>(ws, L.v), at<TX>(ws, L.ell), lse,
         at<float>(ws, L.delta), at<float>(ws, L.dqt), at<float>(ws, L.dkt), at<float>(ws, L.dv),
         n, d, p->causal, scale, scale * ra::kLog2e);
   }
@@ -274,7 +379,8 @@ ra_status simt_bwd(const ra_problem* p, const void* O, const float* lse, float* 
   }
   if (loss) {
     Launch l(K_LOSS, st);
-    loss_finalize_kernel<<<1, 256, 0, st>>>(at<double>(ws, L.loss_part), L.nparts, loss);
+    loss_finalize_kernel<<<1, 256, 0, st>>>(at<double>(ws, L.loss_part),
+                                            holds ? L.nparts_fwd : L.nparts_pre, loss);
   }
   return launch_status();
 }
@@ -300,7 +406,7 @@ ra_status rope_attn_fwd(const ra_problem* p, void* O, float* lse, float* loss, v
   if (s != RA_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (p->dtype == RA_F32) return simt_fwd<float>(p, O, lse, loss, ws, st);
-  return simt_fwd<__nv_bfloat16>(p, O, lse, loss, ws, st);
+  return tc_fwd(p, O, lse, loss, ws, st);
 }
 
 ra_status rope_attn_loss_bwd(const ra_problem* p, const void* O, const float* lse, float* loss,
@@ -317,8 +423,9 @@ ra_status rope_attn_loss_bwd(const ra_problem* p, const void* O, const float* ls
   if (s != RA_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (p->dtype == RA_F32)
-    return simt_bwd<float>(p, O, lse, loss, dWQ, dWK, dWV, ws, ws_holds_fwd, st);
-  return simt_bwd<__nv_bfloat16>(p, O, lse, loss, dWQ, dWK, dWV, ws, ws_holds_fwd, st);
+    return simt_bwd<float, float>(p, O, lse, loss, dWQ, dWK, dWV, ws, ws_holds_fwd, st);
+  return simt_bwd<__nv_bfloat16, __nv_bfloat16>(p, O, lse, loss, dWQ, dWK, dWV, ws, ws_holds_fwd,
+                                                st);
 }
 
 ra_status rope_attn_last_error(void* stream) {

@@ -241,9 +241,10 @@ bwd_pre_kernel(const T* __restrict__ O, const T* __restrict__ E, TL* __restrict_
 //   dV += P^T l,  dK~ += gamma^T Q~ / sqrt(d),  dQ~ += gamma K~ / sqrt(d) (atomic adds)
 // grid (ceil(n/32), B*H), 256 threads, thread (r = tid/8, g = tid%8).
 // ---------------------------------------------------------------------------------------
+template <class TX>
 __global__ void __launch_bounds__(kThreads)
-attn_bwd_kernel(const float* __restrict__ Qt, const float* __restrict__ Kt,
-                const float* __restrict__ V, const float* __restrict__ ell,
+attn_bwd_kernel(const TX* __restrict__ Qt, const TX* __restrict__ Kt,
+                const TX* __restrict__ V, const TX* __restrict__ ell,
                 const float* __restrict__ lse, const float* __restrict__ delta,
                 float* __restrict__ dQt, float* __restrict__ dKt, float* __restrict__ dV,
                 int n, int d, int causal, float scale, float scale_log2) {

@@ -1,0 +1,194 @@
+// Test harness for the sm_100a primitives of librope_attn (tests only).
+//
+// probe_mma: one CTA computes D = A * B with tcgen05 for one operand arrangement (A and B
+//   each K-major or MN-major in 128-byte-swizzled shared memory, or A from TMEM), so each
+//   descriptor form the library uses is checked in isolation against torch.
+// probe_timeout: a kernel waits on an mbarrier that nothing arrives on; the bounded wait
+//   must give up, record a timeout in the status word and return (no trap, no hang).
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../loss_closed_form_b200/csrc/tc_ptx.cuh"
+
+using namespace ra;
+using namespace ra::tc;
+
+namespace {
+
+constexpr int kSmemA = 32768;   // up to 128 x 128 bf16
+constexpr int kSmemB = 65536;   // up to 128 x 256 bf16
+constexpr int kTmemCols = 512;
+
+__global__ void __launch_bounds__(128)
+probe_mma_kernel(const __nv_bfloat16* __restrict__ A, const __nv_bfloat16* __restrict__ B,
+                 float* __restrict__ D, int M, int N, int K, int a_mn, int b_mn, int a_tmem,
+                 unsigned long long limit_ns) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + kSmemA;
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + kSmemA + kSmemB);
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(bar + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tslot + 1);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+  // A into swizzled smem: 16-byte chunks of 8 consecutive elements along the major axis
+  for (int e = tid; e < M * K / 8; e += 128) {
+    uint32_t vals[4];
+    __nv_bfloat16 tmp[8];
+    uint32_t off;
+    if (!a_mn) {  // rows = m, K contiguous
+      const int m = e / (K / 8), k0 = (e % (K / 8)) * 8;
+      for (int i = 0; i < 8; ++i) tmp[i] = A[(size_t)m * K + k0 + i];
+      off = (k0 / 64) * (M * 128) + sw128_offset(m, (k0 % 64) / 8);
+    } else {      // rows = k, M contiguous
+      const int k = e / (M / 8), m0 = (e % (M / 8)) * 8;
+      for (int i = 0; i < 8; ++i) tmp[i] = A[(size_t)(m0 + i) * K + k];
+      off = (m0 / 64) * (K * 128) + sw128_offset(k, (m0 % 64) / 8);
+    }
+    for (int i = 0; i < 4; ++i)
+      vals[i] = (uint32_t)__bfloat16_as_ushort(tmp[2 * i]) |
+                ((uint32_t)__bfloat16_as_ushort(tmp[2 * i + 1]) << 16);
+    st_shared_v4(smem_u32(sA) + off, vals[0], vals[1], vals[2], vals[3]);
+  }
+  for (int e = tid; e < K * N / 8; e += 128) {
+    uint32_t vals[4];
+    __nv_bfloat16 tmp[8];
+    uint32_t off;
+    if (!b_mn) {  // rows = n, K contiguous
+      const int nn = e / (K / 8), k0 = (e % (K / 8)) * 8;
+      for (int i = 0; i < 8; ++i) tmp[i] = B[(size_t)(k0 + i) * N + nn];
+      off = (k0 / 64) * (N * 128) + sw128_offset(nn, (k0 % 64) / 8);
+    } else {      // rows = k, N contiguous
+      const int k = e / (N / 8), n0 = (e % (N / 8)) * 8;
+      for (int i = 0; i < 8; ++i) tmp[i] = B[(size_t)k * N + n0 + i];
+      off = (n0 / 64) * (K * 128) + sw128_offset(k, (n0 % 64) / 8);
+    }
+    for (int i = 0; i < 4; ++i)
+      vals[i] = (uint32_t)__bfloat16_as_ushort(tmp[2 * i]) |
+                ((uint32_t)__bfloat16_as_ushort(tmp[2 * i + 1]) << 16);
+    st_shared_v4(smem_u32(sB) + off, vals[0], vals[1], vals[2], vals[3]);
+  }
+  if (tid == 0) {
+    mbar_init(smem_u32(bar), 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  fence_proxy_async_smem();
+  if (warp == 0) {
+    tmem_alloc(smem_u32(tslot), kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tslot;
+  const uint32_t d_tmem = tmem;        // columns 0 .. N-1
+  const uint32_t a_tm = tmem + 256;    // columns 256 .. 256 + K/2 - 1
+  if (a_tmem) {  // M == 128: row `tid` of A into TMEM lane `tid`, two bf16 per column
+    for (int c0 = 0; c0 < K / 2; c0 += 32) {
+      uint32_t r[32];
+      for (int c = 0; c < 32; ++c)
+        r[c] = (uint32_t)__bfloat16_as_ushort(A[(size_t)tid * K + 2 * (c0 + c)]) |
+               ((uint32_t)__bfloat16_as_ushort(A[(size_t)tid * K + 2 * (c0 + c) + 1]) << 16);
+      tmem_st32(a_tm + ((uint32_t)(warp * 32) << 16) + c0, r);
+    }
+    tmem_wait_st();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (tid == 0) {
+    const uint32_t idesc = idesc_bf16_f32(M, N, a_mn, b_mn);
+    for (int kk = 0; kk < K / 16; ++kk) {
+      uint64_t bd;
+      if (!b_mn)
+        bd = sw128_desc(smem_u32(sB) + (kk / 4) * (N * 128) + (kk % 4) * 32, 16, 1024);
+      else
+        bd = sw128_desc(smem_u32(sB) + kk * 2048, K * 128, 1024);
+      if (a_tmem) {
+        mma_ts(d_tmem, a_tm + kk * 8, bd, idesc, kk > 0);
+      } else {
+        uint64_t ad;
+        if (!a_mn)
+          ad = sw128_desc(smem_u32(sA) + (kk / 4) * (M * 128) + (kk % 4) * 32, 16, 1024);
+        else
+          ad = sw128_desc(smem_u32(sA) + kk * 2048, K * 128, 1024);
+        mma_ss(d_tmem, ad, bd, idesc, kk > 0);
+      }
+    }
+    mma_commit(smem_u32(bar));
+  }
+  __syncwarp();
+  const bool ok = mbar_wait(smem_u32(bar), 0, abort_flag, limit_ns);
+  tc_fence_after();
+  if (ok) {
+    // M = 128: row r in lane r.  M = 64: row r in lane (r % 16) + 32 * (r / 16).
+    const int row = (M == 128) ? tid : (warp * 16 + lane);
+    const bool has_row = (M == 128) || lane < 16;
+    for (int c0 = 0; c0 < N; c0 += 32) {
+      uint32_t r[32];
+      tmem_ld32(d_tmem + ((uint32_t)(warp * 32) << 16) + c0, r);
+      tmem_wait_ld();
+      if (has_row)
+        for (int c = 0; c < 32; ++c) D[(size_t)row * N + c0 + c] = __uint_as_float(r[c]);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+__global__ void probe_timeout_kernel(unsigned long long limit_ns, int* waited_ok) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  // nothing ever arrives on `bar`: the wait must give up after limit_ns
+  const bool ok = mbar_wait(smem_u32(&bar), 0, &abort_flag, limit_ns);
+  if (threadIdx.x == 0) *waited_ok = ok ? 1 : 0;
+}
+
+}  // namespace
+
+extern "C" {
+
+int probe_mma(const void* A, const void* B, float* D, int M, int N, int K, int a_mn, int b_mn,
+              int a_tmem, void* stream) {
+  if (!(M == 64 || M == 128) || !(N == 64 || N == 128 || N == 256) || !(K == 64 || K == 128) ||
+      (a_tmem && (M != 128 || a_mn)))
+    return -1;
+  const int smem = kSmemA + kSmemB + 1024 + 64;
+  cudaFuncSetAttribute(probe_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  probe_mma_kernel<<<1, 128, smem, static_cast<cudaStream_t>(stream)>>>(
+      (const __nv_bfloat16*)A, (const __nv_bfloat16*)B, D, M, N, K, a_mn, b_mn, a_tmem,
+      2000000000ull);
+  return (int)cudaGetLastError();
+}
+
+// Returns the status word after a wait that runs out: 1 (timeout) expected; also whether
+// the wait reported success (must be 0).
+int probe_timeout(unsigned long long limit_ns, int* waited_ok_host) {
+  int* dflag = nullptr;
+  if (cudaMalloc(&dflag, sizeof(int)) != cudaSuccess) return -1;
+  int zero = 0;
+  cudaMemcpyToSymbol(ra::g_status, &zero, sizeof(int));
+  probe_timeout_kernel<<<1, 64>>>(limit_ns, dflag);
+  if (cudaDeviceSynchronize() != cudaSuccess) return -2;
+  int st = 0;
+  cudaMemcpyFromSymbol(&st, ra::g_status, sizeof(int));
+  cudaMemcpy(waited_ok_host, dflag, sizeof(int), cudaMemcpyDeviceToHost);
+  cudaFree(dflag);
+  cudaMemcpyToSymbol(ra::g_status, &zero, sizeof(int));
+  return st;
+}
+
+}  // extern "C"

@@ -1,0 +1,58 @@
+"""Each tcgen05 operand arrangement the kernels use, checked against torch (GPU only)."""
+import ctypes
+
+import pytest
+import torch
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def probe():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from tests_support import probe_lib
+    return probe_lib()
+
+
+CASES = [
+    # M, N, K, a_mn, b_mn, a_tmem
+    (128, 128, 128, 0, 0, 0),   # scores: Q K^T, both K-major
+    (128, 64, 128, 0, 0, 0),    # backward S^T / beta^T tiles (N = 64)
+    (128, 128, 64, 0, 0, 0),
+    (128, 128, 128, 0, 1, 1),   # forward P V: A from TMEM, B MN-major
+    (128, 64, 128, 0, 1, 1),
+    (128, 128, 64, 0, 1, 0),    # backward dV, dK: B MN-major
+    (128, 64, 128, 1, 1, 0),    # backward dQ^T: A MN-major, B MN-major
+    (128, 64, 128, 1, 0, 0),
+    (128, 256, 128, 0, 0, 0),
+    (64, 64, 128, 1, 1, 0),     # weight gradient at d = 64 (M = 64)
+    (64, 128, 64, 0, 0, 0),
+    (128, 128, 128, 1, 1, 0),   # weight gradient at d = 128
+]
+
+
+@pytest.mark.parametrize("M,N,K,a_mn,b_mn,a_tmem", CASES)
+def test_mma_form(probe, M, N, K, a_mn, b_mn, a_tmem):
+    g = torch.Generator(device="cuda").manual_seed(M * 7 + N * 3 + K + a_mn + 2 * b_mn)
+    A = torch.randn(M, K, device="cuda", generator=g).to(torch.bfloat16)
+    B = torch.randn(K, N, device="cuda", generator=g).to(torch.bfloat16)
+    D = torch.full((M, N), float("nan"), device="cuda")
+    rc = probe.probe_mma(ctypes.c_void_p(A.data_ptr()), ctypes.c_void_p(B.data_ptr()),
+                         ctypes.c_void_p(D.data_ptr()), M, N, K, a_mn, b_mn, a_tmem,
+                         ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert rc == 0
+    torch.cuda.synchronize()
+    ref = A.float() @ B.float()
+    err = (D - ref).abs().max().item()
+    assert err <= 1e-3 * ref.abs().max().item(), err
+
+
+def test_bounded_wait_gives_up(probe):
+    ok = ctypes.c_int(7)
+    st = probe.probe_timeout(ctypes.c_ulonglong(20_000_000), ctypes.byref(ok))
+    assert st == 1, st          # timeout recorded in the status word
+    assert ok.value == 0        # the wait reported failure instead of hanging
+    # the context is still usable
+    x = torch.ones(4, device="cuda")
+    assert float(x.sum()) == 4.0
