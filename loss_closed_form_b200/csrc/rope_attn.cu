@@ -17,6 +17,7 @@
 #include "common.cuh"
 #include "simt_kernels.cuh"
 #include "tc_attn_fwd.cuh"
+#include "tc_attn_bwd.cuh"
 
 namespace {
 
@@ -33,12 +34,13 @@ enum KernelId : int {
   K_DW_REDUCE,
   K_LOSS,
   K_FWD_TC,
+  K_BWD_TC,
   K_COUNT
 };
 const char* const kKernelNames[K_COUNT] = {
     "rope_table", "proj_rope_simt", "attn_fwd_simt", "bwd_pre",
     "attn_bwd_simt", "dw_partial_simt", "dw_reduce", "loss_finalize",
-    "attn_fwd_tc"};
+    "attn_fwd_tc", "attn_bwd_tc"};
 
 struct ProfRecord {
   int id;
@@ -332,6 +334,39 @@ ra_status tc_fwd(const ra_problem* p, void* O, float* lse, float* loss, void* ws
   return launch_status();
 }
 
+template <int D>
+ra_status tc_bwd_launch(const ra_problem* p, const Layout& L, const float* lse, void* ws,
+                        cudaStream_t st) {
+  using namespace ra::tc;
+  using C = BwdCfg<D>;
+  const int n = p->n, BH = p->B * p->H;
+  CUtensorMap mq, mk, mv, ml;
+  if (!map_bf16_3d(&mq, at<void>(ws, L.qt), D, n, BH, C::BQ) ||
+      !map_bf16_3d(&mk, at<void>(ws, L.kt), D, n, BH, C::BK) ||
+      !map_bf16_3d(&mv, at<void>(ws, L.v), D, n, BH, C::BK) ||
+      !map_bf16_3d(&ml, at<void>(ws, L.ell), D, n, BH, C::BQ))
+    return RA_ERR_CUDA;
+  BwdParams bp;
+  bp.lse = lse;
+  bp.delta = at<float>(ws, L.delta);
+  bp.dQt = at<float>(ws, L.dqt);
+  bp.dKt = at<float>(ws, L.dkt);
+  bp.dV = at<float>(ws, L.dv);
+  bp.n = n;
+  bp.BH = BH;
+  bp.nk = (n + C::BK - 1) / C::BK;
+  bp.causal = p->causal;
+  bp.scale = 1.0f / sqrtf((float)D);
+  bp.scale_log2 = ra::kLog2e / sqrtf((float)D);
+  bp.limit_ns = wait_limit_ns();
+  auto k = attn_bwd_tc_kernel<D>;
+  cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_ALLOC);
+  dim3 grid(BH, bp.nk);
+  Launch l(K_BWD_TC, st);
+  k<<<grid, C::THREADS, C::SMEM_ALLOC, st>>>(mq, mk, mv, ml, bp);
+  return RA_OK;
+}
+
 template <class T, class TX>
 ra_status simt_bwd(const ra_problem* p, const void* O, const float* lse, float* loss,
                    float* dWQ, float* dWK, float* dWV, void* ws, int holds, cudaStream_t st) {
@@ -351,7 +386,11 @@ ra_status simt_bwd(const ra_problem* p, const void* O, const float* lse, float* 
   if (cudaMemsetAsync(at<float>(ws, L.dqt), 0, act * sizeof(float), st) != cudaSuccess)
     return RA_ERR_CUDA;
   const float scale = 1.0f / sqrtf((float)d);
-  {
+  if constexpr (sizeof(TX) == 2) {
+    ra_status s = d == 128 ? tc_bwd_launch<128>(p, L, lse, ws, st)
+                           : tc_bwd_launch<64>(p, L, lse, ws, st);
+    if (s != RA_OK) return s;
+  } else {
     size_t smem = (size_t)(4 * kRows * (d + 4) + 2 * kRows * 33 + 2 * kRows) * sizeof(float);
     cudaFuncSetAttribute(attn_bwd_kernel<TX>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          (int)smem);

@@ -1,0 +1,378 @@
+// Tensor-core closed-form backward: one CTA per 128-key tile of one (b, h) instance, looping
+// over the 64-row query tiles that see those keys.
+//
+// Per query tile i (all products tcgen05, bf16 operands, fp32 accumulators in TMEM):
+//   S^T    = K~ Q~_i^T                  scores, keys on TMEM lanes
+//   beta^T = V l_i^T                    beta(x) = l V^T, transposed
+//   P^T    = exp(S^T / sqrt(d) - lse_i)  recomputed softmax s(x) from the stored log-sum-exp
+//   gamma^T = P^T o (beta^T - delta_i)   gamma = diag(s) beta - s s^T beta, with the row sums
+//                                        s_i^T beta_i = <l_i, O_i> = delta_i
+//   dV    += P^T l_i                   (accumulated in TMEM over all query tiles)
+//   dK~   += gamma^T Q~_i              (scaled by 1/sqrt(d) at the end)
+//   dQ~_i^T = K~^T gamma^T             (d on TMEM lanes; added to global fp32 dQ~)
+// so no n x n matrix ever leaves the chip.
+//
+// Definitions: "RoPE Attention kan bijna lineair worden getraind", Methodologie 1 (s, l,
+// beta, gamma) and 2 (gamma_1 = diag(s) beta, gamma_2 = s s^T beta).
+//
+// Warp roles (320 threads): warps 0-3 softmax / gamma and the dK, dV epilogue (one key row
+// per thread), warps 4-7 drain dQ~ from TMEM, warp 8 TMA producer (it also stages the
+// query tile's lse and delta), warp 9 MMA issuer and TMEM owner.
+#pragma once
+#include "tc_ptx.cuh"
+
+namespace ra {
+namespace tc {
+
+template <int D>
+struct BwdCfg {
+  static constexpr int BK = 128;              // keys per CTA
+  static constexpr int BQ = 64;               // query rows per step
+  static constexpr int NSQ = 2;               // query-tile pipeline stages
+  static constexpr int KB = D / 64;           // 128-byte swizzle blocks per row
+  static constexpr int KTILE = BK * D * 2;    // K~ or V tile bytes
+  static constexpr int QTILE = BQ * D * 2;    // Q~_i or l_i tile bytes
+  static constexpr int KBLK = BK * 128;       // one swizzle block of a 128-row tile
+  static constexpr int QBLK = BQ * 128;       // one swizzle block of a 64-row tile
+  static constexpr int PG = BK * BQ * 2;      // P^T or gamma^T buffer bytes (one block)
+  static constexpr int K_OFF = 0;
+  static constexpr int V_OFF = K_OFF + KTILE;
+  static constexpr int Q_OFF = V_OFF + KTILE;            // NSQ stages
+  static constexpr int L_OFF = Q_OFF + NSQ * QTILE;      // NSQ stages
+  static constexpr int P_OFF = L_OFF + NSQ * QTILE;      // 2 buffers
+  static constexpr int G_OFF = P_OFF + 2 * PG;           // 2 buffers
+  static constexpr int LSE_OFF = G_OFF + 2 * PG;         // float [NSQ][BQ], lse * log2(e)
+  static constexpr int DEL_OFF = LSE_OFF + NSQ * BQ * 4; // float [NSQ][BQ]
+  static constexpr int BAR_OFF = DEL_OFF + NSQ * BQ * 4;
+  // kv_full, q_full[NSQ], q_empty[NSQ], s_full, s_free, pg_full[2], pg_free[2],
+  // dq_full[2], dq_free[2], acc_done, drain
+  static constexpr int NBAR = 1 + 2 * NSQ + 2 + 8 + 2;
+  static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
+  static constexpr int SMEM_USED = MISC_OFF + 64;
+  static constexpr int SMEM_ALLOC =
+      (SMEM_USED + 1024 > 120 * 1024) ? SMEM_USED + 1024 : 120 * 1024;
+  static constexpr int THREADS = 320;
+  // TMEM columns
+  static constexpr uint32_t T_S = 0, T_B = 64, T_DQ0 = 128, T_DQ1 = 192, T_DK = 256,
+                            T_DV = 256 + D;
+  static constexpr uint32_t T_COLS = 512;
+  static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
+};
+
+struct BwdParams {
+  const float* lse;    // [BH][n]
+  const float* delta;  // [BH][n]
+  float* dQt;          // [BH][n][d], accumulated (must start at zero)
+  float* dKt;          // [BH][n][d]
+  float* dV;           // [BH][n][d]
+  int n, BH, nk, causal;
+  float scale;         // 1 / sqrt(d)
+  float scale_log2;    // log2(e) / sqrt(d)
+  unsigned long long limit_ns;
+};
+
+__device__ __forceinline__ void red_add_f32(float* addr, float v) {
+  asm volatile("red.global.add.f32 [%0], %1;" ::"l"(addr), "f"(v) : "memory");
+}
+
+template <int D>
+__global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
+attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_l,
+                   const BwdParams p) {
+  using C = BwdCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const uint32_t sbase = smem_u32(smem);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(smem + C::MISC_OFF);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::MISC_OFF + 4);
+  float* lse_s = reinterpret_cast<float*>(smem + C::LSE_OFF);
+  float* del_s = reinterpret_cast<float*>(smem + C::DEL_OFF);
+
+  const uint32_t b_kv = smem_u32(&bars[0]);
+  auto b_qfull = [&](int s) { return smem_u32(&bars[1 + s]); };
+  auto b_qempty = [&](int s) { return smem_u32(&bars[1 + C::NSQ + s]); };
+  const uint32_t b_sfull = smem_u32(&bars[1 + 2 * C::NSQ]);
+  const uint32_t b_sfree = smem_u32(&bars[2 + 2 * C::NSQ]);
+  auto b_pgfull = [&](int b) { return smem_u32(&bars[3 + 2 * C::NSQ + b]); };
+  auto b_pgfree = [&](int b) { return smem_u32(&bars[5 + 2 * C::NSQ + b]); };
+  auto b_dqfull = [&](int b) { return smem_u32(&bars[7 + 2 * C::NSQ + b]); };
+  auto b_dqfree = [&](int b) { return smem_u32(&bars[9 + 2 * C::NSQ + b]); };
+  const uint32_t b_acc = smem_u32(&bars[11 + 2 * C::NSQ]);
+  const uint32_t b_drain = smem_u32(&bars[12 + 2 * C::NSQ]);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int bh = blockIdx.x;
+  const int kt = blockIdx.y;  // key tile; tile 0 sees the most query tiles when causal
+  const int n = p.n;
+  const int nqt = (n + C::BQ - 1) / C::BQ;
+  const int i_start = p.causal ? (kt * C::BK) / C::BQ : 0;
+  const int NI = nqt - i_start;
+  const uint64_t lim = p.limit_ns;
+
+  if (tid == 0) {
+    mbar_init(b_kv, 1);
+    for (int s = 0; s < C::NSQ; ++s) {
+      mbar_init(b_qfull(s), 2);  // TMA bytes + the staged lse / delta
+      mbar_init(b_qempty(s), 1);
+    }
+    mbar_init(b_sfull, 1);
+    mbar_init(b_sfree, 128);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(b_pgfull(b), 128);
+      mbar_init(b_pgfree(b), 1);
+      mbar_init(b_dqfull(b), 1);
+      mbar_init(b_dqfree(b), 128);
+    }
+    mbar_init(b_acc, 1);
+    mbar_init(b_drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 9) {
+    tmem_alloc(smem_u32(tslot), C::T_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tslot;
+
+  if (warp == 8) {
+    // ------------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      tma_prefetch(&tm_q);
+      tma_prefetch(&tm_k);
+      tma_prefetch(&tm_v);
+      tma_prefetch(&tm_l);
+      mbar_expect_tx(b_kv, 2 * C::KTILE);
+      for (int b = 0; b < C::KB; ++b) {
+        tma_load_3d(sbase + C::K_OFF + b * C::KBLK, &tm_k, b_kv, 64 * b, kt * C::BK, bh);
+        tma_load_3d(sbase + C::V_OFF + b * C::KBLK, &tm_v, b_kv, 64 * b, kt * C::BK, bh);
+      }
+    }
+    __syncwarp();
+    int last = -1;
+    for (int ii = 0; ii < NI; ++ii) {
+      const int s = ii % C::NSQ;
+      if (!mbar_wait_warp(b_qempty(s), ((ii / C::NSQ) & 1) ^ 1, abort_flag, lim)) break;
+      const int q0 = (i_start + ii) * C::BQ;
+      if (lane == 0) {
+        mbar_expect_tx(b_qfull(s), 2 * C::QTILE);
+        for (int b = 0; b < C::KB; ++b) {
+          tma_load_3d(sbase + C::Q_OFF + s * C::QTILE + b * C::QBLK, &tm_q, b_qfull(s), 64 * b,
+                      q0, bh);
+          tma_load_3d(sbase + C::L_OFF + s * C::QTILE + b * C::QBLK, &tm_l, b_qfull(s), 64 * b,
+                      q0, bh);
+        }
+      }
+#pragma unroll
+      for (int h = 0; h < C::BQ / 32; ++h) {
+        const int c = lane + 32 * h, q = q0 + c;
+        lse_s[s * C::BQ + c] = q < n ? p.lse[(size_t)bh * n + q] * kLog2e : 0.f;
+        del_s[s * C::BQ + c] = q < n ? p.delta[(size_t)bh * n + q] : 0.f;
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(b_qfull(s));
+      last = ii;
+    }
+    if (lane == 0 && *abort_flag) {
+      mbar_drain(b_kv, 0, lim);
+      for (int ii = (last - C::NSQ + 1 > 0 ? last - C::NSQ + 1 : 0); ii <= last; ++ii)
+        mbar_drain(b_qfull(ii % C::NSQ), (ii / C::NSQ) & 1, lim);
+    }
+  } else if (warp == 9) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_sb = idesc_bf16_f32(128, C::BQ, false, false);
+      constexpr uint32_t idesc_kv = idesc_bf16_f32(128, D, false, true);
+      constexpr uint32_t idesc_dq = idesc_bf16_f32(D, C::BQ, true, true);
+      const uint32_t ka = sbase + C::K_OFF, va = sbase + C::V_OFF;
+      bool ok = mbar_wait(b_kv, 0, abort_flag, lim);
+      auto issue_sb = [&](int ii) -> bool {
+        const int s = ii % C::NSQ;
+        if (!mbar_wait(b_qfull(s), (ii / C::NSQ) & 1, abort_flag, lim)) return false;
+        tc_fence_after();
+        const uint32_t qb = sbase + C::Q_OFF + s * C::QTILE;
+        const uint32_t lb = sbase + C::L_OFF + s * C::QTILE;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t ko = (kk >> 2) * C::KBLK + (kk & 3) * 32;
+          const uint32_t qo = (kk >> 2) * C::QBLK + (kk & 3) * 32;
+          mma_ss(tmem + C::T_S, sw128_desc(ka + ko, 16, 1024), sw128_desc(qb + qo, 16, 1024),
+                 idesc_sb, kk > 0);
+          mma_ss(tmem + C::T_B, sw128_desc(va + ko, 16, 1024), sw128_desc(lb + qo, 16, 1024),
+                 idesc_sb, kk > 0);
+        }
+        mma_commit(b_sfull);
+        return true;
+      };
+      tc_fence_after();
+      if (ok) ok = issue_sb(0);
+      for (int ii = 0; ok && ii < NI; ++ii) {
+        if (ii + 1 < NI) {
+          if (!(ok = mbar_wait(b_sfree, ii & 1, abort_flag, lim))) break;
+          if (!(ok = issue_sb(ii + 1))) break;
+        }
+        const int pb = ii & 1, s = ii % C::NSQ;
+        if (!(ok = mbar_wait(b_pgfull(pb), (ii >> 1) & 1, abort_flag, lim))) break;
+        tc_fence_after();
+        const uint32_t pt = sbase + C::P_OFF + pb * C::PG;
+        const uint32_t gt = sbase + C::G_OFF + pb * C::PG;
+        const uint32_t qb = sbase + C::Q_OFF + s * C::QTILE;
+        const uint32_t lb = sbase + C::L_OFF + s * C::QTILE;
+        // dV += P^T l_i, dK += gamma^T Q~_i   (M = 128 keys, N = D, K = 64 queries)
+#pragma unroll
+        for (int kk = 0; kk < C::BQ / 16; ++kk) {
+          mma_ss(tmem + C::T_DV, sw128_desc(pt + kk * 32, 16, 1024),
+                 sw128_desc(lb + kk * 2048, C::QBLK, 1024), idesc_kv, (ii > 0 || kk > 0));
+          mma_ss(tmem + C::T_DK, sw128_desc(gt + kk * 32, 16, 1024),
+                 sw128_desc(qb + kk * 2048, C::QBLK, 1024), idesc_kv, (ii > 0 || kk > 0));
+        }
+        // dQ~_i^T = K~^T gamma^T   (M = D, N = 64 queries, K = 128 keys)
+        if (!(ok = mbar_wait(b_dqfree(pb), ((ii >> 1) & 1) ^ 1, abort_flag, lim))) break;
+        tc_fence_after();
+        const uint32_t dq = tmem + (pb ? C::T_DQ1 : C::T_DQ0);
+#pragma unroll
+        for (int kk = 0; kk < C::BK / 16; ++kk)
+          mma_ss(dq, sw128_desc(ka + kk * 2048, C::KBLK, 1024),
+                 sw128_desc(gt + kk * 2048, C::KBLK, 1024), idesc_dq, kk > 0);
+        mma_commit(b_dqfull(pb));
+        mma_commit(b_pgfree(pb));
+        mma_commit(b_qempty(s));
+      }
+      if (ok) {
+        mma_commit(b_acc);
+      } else {
+        mma_commit(b_drain);
+        mbar_drain(b_drain, 0, lim);
+      }
+    }
+  } else if (warp < 4) {
+    // ------------------------------------------------------------------ P^T, gamma^T
+    const int key = kt * C::BK + tid;
+    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    bool ok = true;
+    for (int ii = 0; ii < NI; ++ii) {
+      const int q0 = (i_start + ii) * C::BQ;
+      const int stg = ii % C::NSQ;
+      // the stage's lse / delta (and S^T, beta^T below) for this query tile
+      if (!(ok = mbar_wait_warp(b_qfull(stg), (ii / C::NSQ) & 1, abort_flag, lim))) break;
+      if (!(ok = mbar_wait_warp(b_sfull, ii & 1, abort_flag, lim))) break;
+      tc_fence_after();
+      uint32_t sr[64], br[64];
+      {
+        uint32_t (&s0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[0]);
+        uint32_t (&s1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[32]);
+        uint32_t (&b0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&br[0]);
+        uint32_t (&b1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&br[32]);
+        tmem_ld32(tmem + lane_base + C::T_S, s0);
+        tmem_ld32(tmem + lane_base + C::T_S + 32, s1);
+        tmem_ld32(tmem + lane_base + C::T_B, b0);
+        tmem_ld32(tmem + lane_base + C::T_B + 32, b1);
+        tmem_wait_ld();
+      }
+      tc_fence_before();
+      mbar_arrive(b_sfree);
+      const int pb = ii & 1;
+      if (!(ok = mbar_wait_warp(b_pgfree(pb), ((ii >> 1) & 1) ^ 1, abort_flag, lim))) break;
+      const uint32_t prow = sbase + C::P_OFF + pb * C::PG;
+      const uint32_t grow = sbase + C::G_OFF + pb * C::PG;
+      const float* ls = lse_s + stg * C::BQ;
+      const float* ds = del_s + stg * C::BQ;
+      const bool full = key < n && q0 + C::BQ <= n && (!p.causal || key <= q0);
+#pragma unroll
+      for (int c8 = 0; c8 < 8; ++c8) {
+        uint32_t pw[4], gw[4];
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+          float pv[2], gv[2];
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int c = c8 * 8 + h * 2 + e;
+            const int q = q0 + c;
+            const bool valid = full || (key < n && q < n && (!p.causal || key <= q));
+            const float pr = valid ? exp2f(__uint_as_float(sr[c]) * p.scale_log2 - ls[c]) : 0.f;
+            pv[e] = pr;
+            gv[e] = pr * (__uint_as_float(br[c]) - ds[c]);
+          }
+          pw[h] = pack_bf16x2(pv[0], pv[1]);
+          gw[h] = pack_bf16x2(gv[0], gv[1]);
+        }
+        const uint32_t off = sw128_offset(tid, c8);
+        st_shared_v4(prow + off, pw[0], pw[1], pw[2], pw[3]);
+        st_shared_v4(grow + off, gw[0], gw[1], gw[2], gw[3]);
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(b_pgfull(pb));
+    }
+    // ---- dK~ = scale * sum gamma^T Q~, dV = sum P^T l: one key row per thread
+    if (ok) ok = mbar_wait_warp(b_acc, 0, abort_flag, lim);
+    if (ok) {
+      tc_fence_after();
+      const size_t ro = ((size_t)bh * n + key) * D;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t rk[32], rv[32];
+        tmem_ld32(tmem + lane_base + C::T_DK + 32 * c, rk);
+        tmem_ld32(tmem + lane_base + C::T_DV + 32 * c, rv);
+        tmem_wait_ld();
+        if (key < n) {
+          float4* dk = reinterpret_cast<float4*>(p.dKt + ro + 32 * c);
+          float4* dv = reinterpret_cast<float4*>(p.dV + ro + 32 * c);
+#pragma unroll
+          for (int v = 0; v < 8; ++v) {
+            dk[v] = make_float4(__uint_as_float(rk[4 * v]) * p.scale,
+                                __uint_as_float(rk[4 * v + 1]) * p.scale,
+                                __uint_as_float(rk[4 * v + 2]) * p.scale,
+                                __uint_as_float(rk[4 * v + 3]) * p.scale);
+            dv[v] = make_float4(__uint_as_float(rv[4 * v]), __uint_as_float(rv[4 * v + 1]),
+                                __uint_as_float(rv[4 * v + 2]), __uint_as_float(rv[4 * v + 3]));
+          }
+        }
+      }
+    }
+  } else {
+    // ------------------------------------------------------------------ dQ~ drain (warps 4-7)
+    const int wq = warp - 4;
+    const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
+    // accumulator row (head-dimension index) held by this lane: M = 128 puts row r in lane r,
+    // M = 64 puts row r in lane (r % 16) + 32 (r / 16)
+    const int drow = (D == 128) ? (wq * 32 + lane) : (wq * 16 + lane);
+    const bool has_row = (D == 128) || lane < 16;
+    for (int ii = 0; ii < NI; ++ii) {
+      const int pb = ii & 1;
+      if (!mbar_wait_warp(b_dqfull(pb), (ii >> 1) & 1, abort_flag, lim)) break;
+      tc_fence_after();
+      uint32_t r0[32], r1[32];
+      const uint32_t dq = tmem + lane_base + (pb ? C::T_DQ1 : C::T_DQ0);
+      tmem_ld32(dq, r0);
+      tmem_ld32(dq + 32, r1);
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(b_dqfree(pb));
+      if (has_row) {
+        const int q0 = (i_start + ii) * C::BQ;
+        float* base = p.dQt + ((size_t)bh * n + q0) * D + drow;
+        const int qn = min(C::BQ, n - q0);
+#pragma unroll
+        for (int c = 0; c < 32; ++c)
+          if (c < qn) red_add_f32(base + (size_t)c * D, __uint_as_float(r0[c]) * p.scale);
+#pragma unroll
+        for (int c = 0; c < 32; ++c)
+          if (32 + c < qn) red_add_f32(base + (size_t)(32 + c) * D, __uint_as_float(r1[c]) * p.scale);
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::T_COLS);
+  }
+}
+
+}  // namespace tc
+}  // namespace ra
