@@ -18,6 +18,7 @@
 #include "simt_kernels.cuh"
 #include "tc_attn_fwd.cuh"
 #include "tc_attn_bwd.cuh"
+#include "tc_proj_dw.cuh"
 
 namespace {
 
@@ -35,12 +36,15 @@ enum KernelId : int {
   K_LOSS,
   K_FWD_TC,
   K_BWD_TC,
+  K_PROJ_TC,
+  K_DQ_UNROT,
+  K_DW_TC,
   K_COUNT
 };
 const char* const kKernelNames[K_COUNT] = {
     "rope_table", "proj_rope_simt", "attn_fwd_simt", "bwd_pre",
     "attn_bwd_simt", "dw_partial_simt", "dw_reduce", "loss_finalize",
-    "attn_fwd_tc", "attn_bwd_tc"};
+    "attn_fwd_tc", "attn_bwd_tc", "proj_rope_tc", "dq_unrotate", "dw_tc"};
 
 struct ProfRecord {
   int id;
@@ -98,15 +102,18 @@ struct Layout {
   size_t qt, kt, v;  // intermediate [B][H][n][d] (element size `inter`)
   size_t ell;        // intermediate [B][H][n][d]
   size_t delta;      // float [B][H][n]
-  size_t dqt;        // float [B][H][n][d]
-  size_t dkt;        // float [B][H][n][d]
-  size_t dv;         // float [B][H][n][d]
+  size_t dqt;        // float [B][H][n][d]: gradient w.r.t. Q~ (accumulated)
+  size_t dkt;        // float [B][H][n][d] (fp32 path): gradient w.r.t. K~
+  size_t dv;         // float [B][H][n][d] (fp32 path)
+  size_t dq16;       // bf16 [B][H][n][d] (bf16 path): rot^-1(dQ~)
+  size_t dk16;       // bf16 [B][H][n][d] (bf16 path): rot^-1(dK~)
+  size_t dv16;       // bf16 [B][H][n][d] (bf16 path)
   size_t dw_part;    // float [3][H][nsplit][d][d]
   size_t loss_part;  // double [nparts]
   size_t total;
   int inter;         // bytes per intermediate element
   int nsplit;        // weight-gradient row splits per head
-  int chunk;         // rows per split
+  int chunk;         // rows per split (fp32 path) or 128-row tiles per split (bf16 path)
   int nparts;        // capacity of the loss partial sums
   int nparts_fwd;    // partial sums the forward writes
   int nparts_pre;    // partial sums the backward's own l = O - E pass writes
@@ -138,12 +145,22 @@ Layout make_layout(const ra_problem* p) {
   L.inter = p->dtype == RA_BF16 ? 2 : 4;
   const size_t act = B * H * n * d;
   const long rows = (long)B * n;
-  long ns = (4 * 148 + 3 * p->H - 1) / (3 * p->H);
-  ns = ns < 1 ? 1 : ns;
-  long maxs = (rows + 63) / 64;
-  if (ns > maxs) ns = maxs;
-  L.nsplit = (int)ns;
-  L.chunk = (int)((rows + ns - 1) / ns);
+  if (p->dtype == RA_BF16) {
+    // tensor-core weight gradients: splits of whole 128-row tiles, about two CTAs per SM
+    const long tiles = (long)B * ((n + 127) / 128);
+    long ns = (2 * 148 + 3 * p->H - 1) / (3 * p->H);
+    ns = ns < 1 ? 1 : (ns > tiles ? tiles : ns);
+    const long per = (tiles + ns - 1) / ns;
+    L.chunk = (int)per;                      // tiles per split
+    L.nsplit = (int)((tiles + per - 1) / per);
+  } else {
+    long ns = (4 * 148 + 3 * p->H - 1) / (3 * p->H);
+    ns = ns < 1 ? 1 : ns;
+    long maxs = (rows + 63) / 64;
+    if (ns > maxs) ns = maxs;
+    L.nsplit = (int)ns;
+    L.chunk = (int)((rows + ns - 1) / ns);
+  }
   L.nparts_pre = (int)(((n + 31) / 32) * B * H);
   L.nparts_fwd = p->dtype == RA_BF16 ? (int)(((n + 127) / 128) * B * H) : L.nparts_pre;
   L.nparts = L.nparts_pre;
@@ -159,9 +176,13 @@ Layout make_layout(const ra_problem* p) {
   L.v = take(act * L.inter);
   L.ell = take(act * L.inter);
   L.delta = take(B * H * n * sizeof(float));
+  const bool tcp = p->dtype == RA_BF16;
   L.dqt = take(act * sizeof(float));
-  L.dkt = take(act * sizeof(float));
-  L.dv = take(act * sizeof(float));
+  L.dkt = take(tcp ? 0 : act * sizeof(float));
+  L.dv = take(tcp ? 0 : act * sizeof(float));
+  L.dq16 = take(tcp ? act * 2 : 0);
+  L.dk16 = take(tcp ? act * 2 : 0);
+  L.dv16 = take(tcp ? act * 2 : 0);
   L.dw_part = take(3 * H * (size_t)L.nsplit * d * d * sizeof(float));
   L.loss_part = take((size_t)L.nparts * sizeof(double));
   L.total = off;
@@ -287,6 +308,84 @@ ra_status simt_fwd(const ra_problem* p, void* O, float* lse, float* loss, void* 
 // bf16 tensor-core path
 // ---------------------------------------------------------------------------------------
 template <int D>
+ra_status tc_project(const ra_problem* p, const Layout& L, void* ws, cudaStream_t st) {
+  using namespace ra::tc;
+  using C = ProjCfg<D>;
+  const int n = p->n, BH = p->B * p->H, half = D / 2;
+  float2* tab = at<float2>(ws, L.rope);
+  {
+    int total = n * half;
+    Launch l(K_ROPE_TABLE, st);
+    ra::simt::rope_table_kernel<<<(total + 255) / 256, 256, 0, st>>>(tab, p->pos, n, half,
+                                                                     p->rope_base);
+  }
+  CUtensorMap a1, a2, a3, w1, w2, w3;
+  if (!map_bf16_3d(&a1, p->A1, D, n, BH, C::BM) || !map_bf16_3d(&a2, p->A2, D, n, BH, C::BM) ||
+      !map_bf16_3d(&a3, p->A3, D, n, BH, C::BM) || !map_bf16_3d(&w1, p->WQ, D, D, p->H, D) ||
+      !map_bf16_3d(&w2, p->WK, D, D, p->H, D) || !map_bf16_3d(&w3, p->WV, D, D, p->H, D))
+    return RA_ERR_CUDA;
+  ProjParams pp;
+  pp.tab = tab;
+  pp.out[0] = at<__nv_bfloat16>(ws, L.qt);
+  pp.out[1] = at<__nv_bfloat16>(ws, L.kt);
+  pp.out[2] = at<__nv_bfloat16>(ws, L.v);
+  pp.n = n;
+  pp.H = p->H;
+  pp.limit_ns = wait_limit_ns();
+  auto k = proj_rope_tc_kernel<D>;
+  cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_ALLOC);
+  dim3 grid(BH, (n + C::BM - 1) / C::BM, 3);
+  Launch l(K_PROJ_TC, st);
+  k<<<grid, C::THREADS, C::SMEM_ALLOC, st>>>(a1, a2, a3, w1, w2, w3, pp);
+  return launch_status();
+}
+
+template <int D>
+ra_status tc_weight_grads(const ra_problem* p, const Layout& L, float* dWQ, float* dWK,
+                          float* dWV, void* ws, cudaStream_t st) {
+  using namespace ra::tc;
+  using C = DwCfg<D>;
+  const int n = p->n, BH = p->B * p->H, half = D / 2;
+  {
+    const long long pairs = (long long)BH * n * half;
+    Launch l(K_DQ_UNROT, st);
+    dq_unrotate_kernel<<<(unsigned)((pairs + 255) / 256), 256, 0, st>>>(
+        at<float2>(ws, L.dqt), at<float2>(ws, L.rope), at<__nv_bfloat162>(ws, L.dq16), pairs, n,
+        half);
+  }
+  CUtensorMap a1, a2, a3, x1, x2, x3;
+  if (!map_bf16_3d(&a1, p->A1, D, n, BH, C::BR) || !map_bf16_3d(&a2, p->A2, D, n, BH, C::BR) ||
+      !map_bf16_3d(&a3, p->A3, D, n, BH, C::BR) ||
+      !map_bf16_3d(&x1, at<void>(ws, L.dq16), D, n, BH, C::BR) ||
+      !map_bf16_3d(&x2, at<void>(ws, L.dk16), D, n, BH, C::BR) ||
+      !map_bf16_3d(&x3, at<void>(ws, L.dv16), D, n, BH, C::BR))
+    return RA_ERR_CUDA;
+  DwParams dp;
+  dp.part = at<float>(ws, L.dw_part);
+  dp.n = n;
+  dp.B = p->B;
+  dp.H = p->H;
+  dp.nt = (n + C::BR - 1) / C::BR;
+  dp.nsplit = L.nsplit;
+  dp.tiles_per_split = L.chunk;
+  dp.limit_ns = wait_limit_ns();
+  auto k = dw_tc_kernel<D>;
+  cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_ALLOC);
+  {
+    dim3 grid(L.nsplit, 3, p->H);
+    Launch l(K_DW_TC, st);
+    k<<<grid, C::THREADS, C::SMEM_ALLOC, st>>>(a1, a2, a3, x1, x2, x3, dp);
+  }
+  {
+    size_t total = (size_t)3 * p->H * D * D;
+    Launch l(K_DW_REDUCE, st);
+    ra::simt::dw_reduce_kernel<<<(unsigned)((total + 255) / 256), 256, 0, st>>>(
+        at<float>(ws, L.dw_part), dWQ, dWK, dWV, p->H, D, L.nsplit);
+  }
+  return launch_status();
+}
+
+template <int D>
 ra_status tc_fwd_launch(const ra_problem* p, const Layout& L, void* O, float* lse, void* ws,
                         cudaStream_t st) {
   using namespace ra::tc;
@@ -321,7 +420,7 @@ ra_status tc_fwd_launch(const ra_problem* p, const Layout& L, void* O, float* ls
 ra_status tc_fwd(const ra_problem* p, void* O, float* lse, float* loss, void* ws,
                  cudaStream_t st) {
   const Layout L = make_layout(p);
-  ra_status s = simt_project<__nv_bfloat16, __nv_bfloat16>(p, L, ws, st);
+  ra_status s = p->d == 128 ? tc_project<128>(p, L, ws, st) : tc_project<64>(p, L, ws, st);
   if (s != RA_OK) return s;
   s = p->d == 128 ? tc_fwd_launch<128>(p, L, O, lse, ws, st)
                   : tc_fwd_launch<64>(p, L, O, lse, ws, st);
@@ -349,9 +448,10 @@ ra_status tc_bwd_launch(const ra_problem* p, const Layout& L, const float* lse, 
   BwdParams bp;
   bp.lse = lse;
   bp.delta = at<float>(ws, L.delta);
+  bp.tab = at<float2>(ws, L.rope);
   bp.dQt = at<float>(ws, L.dqt);
-  bp.dKt = at<float>(ws, L.dkt);
-  bp.dV = at<float>(ws, L.dv);
+  bp.dK = at<__nv_bfloat16>(ws, L.dk16);
+  bp.dV = at<__nv_bfloat16>(ws, L.dv16);
   bp.n = n;
   bp.BH = BH;
   bp.nk = (n + C::BK - 1) / C::BK;
@@ -367,37 +467,33 @@ ra_status tc_bwd_launch(const ra_problem* p, const Layout& L, const float* lse, 
   return RA_OK;
 }
 
-template <class T, class TX>
+// fp32 I/O: CUDA-core backward.
 ra_status simt_bwd(const ra_problem* p, const void* O, const float* lse, float* loss,
                    float* dWQ, float* dWK, float* dWV, void* ws, int holds, cudaStream_t st) {
   using namespace ra::simt;
   const Layout L = make_layout(p);
   const int n = p->n, d = p->d;
   if (!holds) {
-    ra_status s = simt_project<T, TX>(p, L, ws, st);
+    ra_status s = simt_project<float, float>(p, L, ws, st);
     if (s != RA_OK) return s;
     dim3 grid((n + kRows - 1) / kRows, p->B * p->H);
     Launch l(K_BWD_PRE, st);
-    bwd_pre_kernel<T, TX><<<grid, kThreads, 0, st>>>(
-        (const T*)O, (const T*)p->E, at<TX>(ws, L.ell), at<float>(ws, L.delta),
+    bwd_pre_kernel<float, float><<<grid, kThreads, 0, st>>>(
+        (const float*)O, (const float*)p->E, at<float>(ws, L.ell), at<float>(ws, L.delta),
         at<double>(ws, L.loss_part), n, d);
   }
   const size_t act = (size_t)p->B * p->H * n * d;
   if (cudaMemsetAsync(at<float>(ws, L.dqt), 0, act * sizeof(float), st) != cudaSuccess)
     return RA_ERR_CUDA;
   const float scale = 1.0f / sqrtf((float)d);
-  if constexpr (sizeof(TX) == 2) {
-    ra_status s = d == 128 ? tc_bwd_launch<128>(p, L, lse, ws, st)
-                           : tc_bwd_launch<64>(p, L, lse, ws, st);
-    if (s != RA_OK) return s;
-  } else {
+  {
     size_t smem = (size_t)(4 * kRows * (d + 4) + 2 * kRows * 33 + 2 * kRows) * sizeof(float);
-    cudaFuncSetAttribute(attn_bwd_kernel<TX>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaFuncSetAttribute(attn_bwd_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          (int)smem);
     dim3 grid((n + kRows - 1) / kRows, p->B * p->H);
     Launch l(K_BWD_SIMT, st);
-    attn_bwd_kernel<TX><<<grid, kThreads, smem, st>>>(
-        at<TX>(ws, L.qt), at<TX>(ws, L.kt), at<TX>(ws, L.v), at<TX>(ws, L.ell), lse,
+    attn_bwd_kernel<float><<<grid, kThreads, smem, st>>>(
+        at<float>(ws, L.qt), at<float>(ws, L.kt), at<float>(ws, L.v), at<float>(ws, L.ell), lse,
         at<float>(ws, L.delta), at<float>(ws, L.dqt), at<float>(ws, L.dkt), at<float>(ws, L.dv),
         n, d, p->causal, scale, scale * ra::kLog2e);
   }
@@ -406,8 +502,8 @@ ra_status simt_bwd(const ra_problem* p, const void* O, const float* lse, float* 
     dim3 grid(L.nsplit, 3, p->H);
     {
       Launch l(K_DW_PART_SIMT, st);
-      dw_partial_kernel<T, float><<<grid, kThreads, smem, st>>>(
-          (const T*)p->A1, (const T*)p->A2, (const T*)p->A3, at<float>(ws, L.dqt),
+      dw_partial_kernel<float, float><<<grid, kThreads, smem, st>>>(
+          (const float*)p->A1, (const float*)p->A2, (const float*)p->A3, at<float>(ws, L.dqt),
           at<float>(ws, L.dkt), at<float>(ws, L.dv), at<float2>(ws, L.rope),
           at<float>(ws, L.dw_part), p->B, p->H, n, d, L.chunk);
     }
@@ -420,6 +516,37 @@ ra_status simt_bwd(const ra_problem* p, const void* O, const float* lse, float* 
     Launch l(K_LOSS, st);
     loss_finalize_kernel<<<1, 256, 0, st>>>(at<double>(ws, L.loss_part),
                                             holds ? L.nparts_fwd : L.nparts_pre, loss);
+  }
+  return launch_status();
+}
+
+// bf16 I/O: tensor-core backward.
+ra_status tc_bwd(const ra_problem* p, const void* O, const float* lse, float* loss, float* dWQ,
+                 float* dWK, float* dWV, void* ws, int holds, cudaStream_t st) {
+  const Layout L = make_layout(p);
+  const int n = p->n, d = p->d;
+  ra_status s;
+  if (!holds) {
+    s = d == 128 ? tc_project<128>(p, L, ws, st) : tc_project<64>(p, L, ws, st);
+    if (s != RA_OK) return s;
+    dim3 grid((n + ra::simt::kRows - 1) / ra::simt::kRows, p->B * p->H);
+    Launch l(K_BWD_PRE, st);
+    ra::simt::bwd_pre_kernel<__nv_bfloat16, __nv_bfloat16><<<grid, ra::simt::kThreads, 0, st>>>(
+        (const __nv_bfloat16*)O, (const __nv_bfloat16*)p->E, at<__nv_bfloat16>(ws, L.ell),
+        at<float>(ws, L.delta), at<double>(ws, L.loss_part), n, d);
+  }
+  const size_t act = (size_t)p->B * p->H * n * d;
+  if (cudaMemsetAsync(at<float>(ws, L.dqt), 0, act * sizeof(float), st) != cudaSuccess)
+    return RA_ERR_CUDA;
+  s = d == 128 ? tc_bwd_launch<128>(p, L, lse, ws, st) : tc_bwd_launch<64>(p, L, lse, ws, st);
+  if (s != RA_OK) return s;
+  s = d == 128 ? tc_weight_grads<128>(p, L, dWQ, dWK, dWV, ws, st)
+               : tc_weight_grads<64>(p, L, dWQ, dWK, dWV, ws, st);
+  if (s != RA_OK) return s;
+  if (loss) {
+    Launch l(K_LOSS, st);
+    ra::simt::loss_finalize_kernel<<<1, 256, 0, st>>>(at<double>(ws, L.loss_part),
+                                                      holds ? L.nparts_fwd : L.nparts_pre, loss);
   }
   return launch_status();
 }
@@ -462,9 +589,8 @@ ra_status rope_attn_loss_bwd(const ra_problem* p, const void* O, const float* ls
   if (s != RA_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (p->dtype == RA_F32)
-    return simt_bwd<float, float>(p, O, lse, loss, dWQ, dWK, dWV, ws, ws_holds_fwd, st);
-  return simt_bwd<__nv_bfloat16, __nv_bfloat16>(p, O, lse, loss, dWQ, dWK, dWV, ws, ws_holds_fwd,
-                                                st);
+    return simt_bwd(p, O, lse, loss, dWQ, dWK, dWV, ws, ws_holds_fwd, st);
+  return tc_bwd(p, O, lse, loss, dWQ, dWK, dWV, ws, ws_holds_fwd, st);
 }
 
 ra_status rope_attn_last_error(void* stream) {

@@ -8,7 +8,7 @@
 //   gamma^T = P^T o (beta^T - delta_i)   gamma = diag(s) beta - s s^T beta, with the row sums
 //                                        s_i^T beta_i = <l_i, O_i> = delta_i
 //   dV    += P^T l_i                   (accumulated in TMEM over all query tiles)
-//   dK~   += gamma^T Q~_i              (scaled by 1/sqrt(d) at the end)
+//   dK~   += gamma^T Q~_i              (scaled by 1/sqrt(d) and un-rotated at the end)
 //   dQ~_i^T = K~^T gamma^T             (d on TMEM lanes; added to global fp32 dQ~)
 // so no n x n matrix ever leaves the chip.
 //
@@ -60,11 +60,12 @@ struct BwdCfg {
 };
 
 struct BwdParams {
-  const float* lse;    // [BH][n]
-  const float* delta;  // [BH][n]
-  float* dQt;          // [BH][n][d], accumulated (must start at zero)
-  float* dKt;          // [BH][n][d]
-  float* dV;           // [BH][n][d]
+  const float* lse;     // [BH][n]
+  const float* delta;   // [BH][n]
+  const float2* tab;    // [n][d/2] (cos, sin) of the RoPE angles
+  float* dQt;           // [BH][n][d] gradient w.r.t. Q~, accumulated (must start at zero)
+  __nv_bfloat16* dK;    // [BH][n][d] rot^-1(dK~), bf16
+  __nv_bfloat16* dV;    // [BH][n][d] bf16
   int n, BH, nk, causal;
   float scale;         // 1 / sqrt(d)
   float scale_log2;    // log2(e) / sqrt(d)
@@ -308,11 +309,12 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       fence_proxy_async_smem();
       mbar_arrive(b_pgfull(pb));
     }
-    // ---- dK~ = scale * sum gamma^T Q~, dV = sum P^T l: one key row per thread
+    // ---- dK = rot^-1(scale * sum gamma^T Q~), dV = sum P^T l: one key row per thread
     if (ok) ok = mbar_wait_warp(b_acc, 0, abort_flag, lim);
     if (ok) {
       tc_fence_after();
       const size_t ro = ((size_t)bh * n + key) * D;
+      const float2* tr = p.tab + (size_t)(key < n ? key : 0) * (D / 2);
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t rk[32], rv[32];
@@ -320,16 +322,21 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         tmem_ld32(tmem + lane_base + C::T_DV + 32 * c, rv);
         tmem_wait_ld();
         if (key < n) {
-          float4* dk = reinterpret_cast<float4*>(p.dKt + ro + 32 * c);
-          float4* dv = reinterpret_cast<float4*>(p.dV + ro + 32 * c);
+          uint32_t wk[16], wv[16];
 #pragma unroll
-          for (int v = 0; v < 8; ++v) {
-            dk[v] = make_float4(__uint_as_float(rk[4 * v]) * p.scale,
-                                __uint_as_float(rk[4 * v + 1]) * p.scale,
-                                __uint_as_float(rk[4 * v + 2]) * p.scale,
-                                __uint_as_float(rk[4 * v + 3]) * p.scale);
-            dv[v] = make_float4(__uint_as_float(rv[4 * v]), __uint_as_float(rv[4 * v + 1]),
-                                __uint_as_float(rv[4 * v + 2]), __uint_as_float(rv[4 * v + 3]));
+          for (int k = 0; k < 16; ++k) {
+            const float x0 = __uint_as_float(rk[2 * k]) * p.scale;
+            const float x1 = __uint_as_float(rk[2 * k + 1]) * p.scale;
+            const float2 cs = tr[16 * c + k];  // rotation by -phi
+            wk[k] = pack_bf16x2(x0 * cs.x + x1 * cs.y, -x0 * cs.y + x1 * cs.x);
+            wv[k] = pack_bf16x2(__uint_as_float(rv[2 * k]), __uint_as_float(rv[2 * k + 1]));
+          }
+          uint4* dk = reinterpret_cast<uint4*>(p.dK + ro + 32 * c);
+          uint4* dv = reinterpret_cast<uint4*>(p.dV + ro + 32 * c);
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            dk[v] = make_uint4(wk[4 * v], wk[4 * v + 1], wk[4 * v + 2], wk[4 * v + 3]);
+            dv[v] = make_uint4(wv[4 * v], wv[4 * v + 1], wv[4 * v + 2], wv[4 * v + 3]);
           }
         }
       }
