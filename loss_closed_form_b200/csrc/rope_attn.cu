@@ -411,7 +411,7 @@ ra_status tc_fwd_launch(const ra_problem* p, const Layout& L, void* O, float* ls
   fp.limit_ns = wait_limit_ns();
   auto k = attn_fwd_tc_kernel<D>;
   cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_ALLOC);
-  dim3 grid(BH, fp.nq);
+  dim3 grid(fp.nq, BH);
   Launch l(K_FWD_TC, st);
   k<<<grid, C::THREADS, C::SMEM_ALLOC, st>>>(mq, mk, mv, fp);
   return RA_OK;
@@ -461,7 +461,7 @@ ra_status tc_bwd_launch(const ra_problem* p, const Layout& L, const float* lse, 
   bp.limit_ns = wait_limit_ns();
   auto k = attn_bwd_tc_kernel<D>;
   cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_ALLOC);
-  dim3 grid(BH, bp.nk);
+  dim3 grid(bp.nk, BH);
   Launch l(K_BWD_TC, st);
   k<<<grid, C::THREADS, C::SMEM_ALLOC, st>>>(mq, mk, mv, ml, bp);
   return RA_OK;

@@ -41,9 +41,9 @@ struct BwdCfg {
   static constexpr int L_OFF = Q_OFF + NSQ * QTILE;      // NSQ stages
   static constexpr int P_OFF = L_OFF + NSQ * QTILE;      // 2 buffers
   static constexpr int G_OFF = P_OFF + 2 * PG;           // 2 buffers
-  static constexpr int LSE_OFF = G_OFF + 2 * PG;         // float [NSQ][BQ], lse * log2(e)
-  static constexpr int DEL_OFF = LSE_OFF + NSQ * BQ * 4; // float [NSQ][BQ]
-  static constexpr int BAR_OFF = DEL_OFF + NSQ * BQ * 4;
+  // float [NSQ][BQ][2]: (lse * log2(e), delta) per query row
+  static constexpr int LD_OFF = G_OFF + 2 * PG;
+  static constexpr int BAR_OFF = LD_OFF + NSQ * BQ * 8;
   // kv_full, q_full[NSQ], q_empty[NSQ], s_full, s_free, pg_full[2], pg_free[2],
   // dq_full[2], dq_free[2], acc_done, drain
   static constexpr int NBAR = 1 + 2 * NSQ + 2 + 8 + 2;
@@ -89,8 +89,7 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
   uint32_t* tslot = reinterpret_cast<uint32_t*>(smem + C::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::MISC_OFF + 4);
-  float* lse_s = reinterpret_cast<float*>(smem + C::LSE_OFF);
-  float* del_s = reinterpret_cast<float*>(smem + C::DEL_OFF);
+  float2* ld_s = reinterpret_cast<float2*>(smem + C::LD_OFF);
 
   const uint32_t b_kv = smem_u32(&bars[0]);
   auto b_qfull = [&](int s) { return smem_u32(&bars[1 + s]); };
@@ -105,8 +104,10 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
   const uint32_t b_drain = smem_u32(&bars[12 + 2 * C::NSQ]);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int bh = blockIdx.x;
-  const int kt = blockIdx.y;  // key tile; tile 0 sees the most query tiles when causal
+  // head-major order: the key tiles of one (b, h) run side by side and share its Q~, l and
+  // dQ~ in L2; key tile 0 sees the most query tiles when causal, so it goes first
+  const int kt = blockIdx.x;
+  const int bh = blockIdx.y;
   const int n = p.n;
   const int nqt = (n + C::BQ - 1) / C::BQ;
   const int i_start = p.causal ? (kt * C::BK) / C::BQ : 0;
@@ -172,8 +173,9 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
 #pragma unroll
       for (int h = 0; h < C::BQ / 32; ++h) {
         const int c = lane + 32 * h, q = q0 + c;
-        lse_s[s * C::BQ + c] = q < n ? p.lse[(size_t)bh * n + q] * kLog2e : 0.f;
-        del_s[s * C::BQ + c] = q < n ? p.delta[(size_t)bh * n + q] : 0.f;
+        ld_s[s * C::BQ + c] = q < n ? make_float2(p.lse[(size_t)bh * n + q] * kLog2e,
+                                                  p.delta[(size_t)bh * n + q])
+                                    : make_float2(0.f, 0.f);
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(b_qfull(s));
@@ -281,26 +283,23 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       if (!(ok = mbar_wait_warp(b_pgfree(pb), ((ii >> 1) & 1) ^ 1, abort_flag, lim))) break;
       const uint32_t prow = sbase + C::P_OFF + pb * C::PG;
       const uint32_t grow = sbase + C::G_OFF + pb * C::PG;
-      const float* ls = lse_s + stg * C::BQ;
-      const float* ds = del_s + stg * C::BQ;
+      const float4* ld4 = reinterpret_cast<const float4*>(ld_s + stg * C::BQ);
       const bool full = key < n && q0 + C::BQ <= n && (!p.causal || key <= q0);
 #pragma unroll
       for (int c8 = 0; c8 < 8; ++c8) {
         uint32_t pw[4], gw[4];
 #pragma unroll
         for (int h = 0; h < 4; ++h) {
-          float pv[2], gv[2];
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int c = c8 * 8 + h * 2 + e;
-            const int q = q0 + c;
-            const bool valid = full || (key < n && q < n && (!p.causal || key <= q));
-            const float pr = valid ? exp2f(__uint_as_float(sr[c]) * p.scale_log2 - ls[c]) : 0.f;
-            pv[e] = pr;
-            gv[e] = pr * (__uint_as_float(br[c]) - ds[c]);
-          }
-          pw[h] = pack_bf16x2(pv[0], pv[1]);
-          gw[h] = pack_bf16x2(gv[0], gv[1]);
+          const int c = c8 * 8 + h * 2;
+          const float4 lz = ld4[c >> 1];  // (lse_c, delta_c, lse_c+1, delta_c+1)
+          const int q = q0 + c;
+          const bool v0 = full || (key < n && q < n && (!p.causal || key <= q));
+          const bool v1 = full || (key < n && q + 1 < n && (!p.causal || key <= q + 1));
+          const float p0 = v0 ? ex2(__uint_as_float(sr[c]) * p.scale_log2 - lz.x) : 0.f;
+          const float p1 = v1 ? ex2(__uint_as_float(sr[c + 1]) * p.scale_log2 - lz.z) : 0.f;
+          pw[h] = pack_bf16x2(p0, p1);
+          gw[h] = pack_bf16x2(p0 * (__uint_as_float(br[c]) - lz.y),
+                              p1 * (__uint_as_float(br[c + 1]) - lz.w));
         }
         const uint32_t off = sw128_offset(tid, c8);
         st_shared_v4(prow + off, pw[0], pw[1], pw[2], pw[3]);

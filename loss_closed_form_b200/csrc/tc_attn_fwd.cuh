@@ -85,8 +85,10 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
   const uint32_t b_drain = smem_u32(&bars[7 + 4 * C::NS]);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int bh = blockIdx.x;
-  const int qt = p.nq - 1 - blockIdx.y;  // longest causal tiles first
+  // head-major order: the query tiles of one (b, h) run side by side and share its K~, V in
+  // L2; within a head the longest causal tiles go first
+  const int bh = blockIdx.y;
+  const int qt = p.nq - 1 - blockIdx.x;
   const int n = p.n;
   const int T = p.causal ? qt + 1 : (n + C::BN - 1) / C::BN;
   const uint64_t lim = p.limit_ns;
@@ -261,7 +263,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
       uint32_t pk[64];
 #pragma unroll
       for (int i = 0; i < 64; ++i) {
-        const float p0 = exp2f(x[2 * i] - m), p1 = exp2f(x[2 * i + 1] - m);
+        const float p0 = ex2(x[2 * i] - m), p1 = ex2(x[2 * i + 1] - m);
         psum += p0 + p1;
         pk[i] = pack_bf16x2(p0, p1);
       }
