@@ -9,15 +9,17 @@
 //                                        s_i^T beta_i = <l_i, O_i> = delta_i
 //   dV    += P^T l_i                   (accumulated in TMEM over all query tiles)
 //   dK~   += gamma^T Q~_i              (scaled by 1/sqrt(d) and un-rotated at the end)
-//   dQ~_i^T = K~^T gamma^T             (d on TMEM lanes; added to global fp32 dQ~)
+//   dQ~_i^T = K~^T gamma^T             (d on TMEM lanes; staged in shared memory and added to
+//                                        the global fp32 dQ~ by one TMA bulk reduce-add)
 // so no n x n matrix ever leaves the chip.
 //
 // Definitions: "RoPE Attention kan bijna lineair worden getraind", Methodologie 1 (s, l,
 // beta, gamma) and 2 (gamma_1 = diag(s) beta, gamma_2 = s s^T beta).
 //
 // Warp roles (320 threads): warps 0-3 softmax / gamma and the dK, dV epilogue (one key row
-// per thread), warps 4-7 drain dQ~ from TMEM, warp 8 TMA producer (it also stages the
-// query tile's lse and delta), warp 9 MMA issuer and TMEM owner.
+// per thread), warps 4-7 drain dQ~ from TMEM into the staging tile (thread 128 issues the
+// bulk reduction), warp 8 TMA producer (it also stages the query tile's lse and delta),
+// warp 9 MMA issuer and TMEM owner.
 #pragma once
 #include "tc_ptx.cuh"
 
@@ -41,12 +43,14 @@ struct BwdCfg {
   static constexpr int L_OFF = Q_OFF + NSQ * QTILE;      // NSQ stages
   static constexpr int P_OFF = L_OFF + NSQ * QTILE;      // 2 buffers
   static constexpr int G_OFF = P_OFF + 2 * PG;           // 2 buffers
+  static constexpr int DQS_OFF = G_OFF + 2 * PG;          // fp32 [BQ][D] dQ~ staging tile
+  static constexpr int DQS = BQ * D * 4;
   // float [NSQ][BQ][2]: (lse * log2(e), delta) per query row
-  static constexpr int LD_OFF = G_OFF + 2 * PG;
+  static constexpr int LD_OFF = DQS_OFF + DQS;
   static constexpr int BAR_OFF = LD_OFF + NSQ * BQ * 8;
   // kv_full, q_full[NSQ], q_empty[NSQ], s_full, s_free, pg_full[2], pg_free[2],
-  // dq_full[2], dq_free[2], acc_done, drain
-  static constexpr int NBAR = 1 + 2 * NSQ + 2 + 8 + 2;
+  // dq_full[2], dq_free[2], acc_done, drain, dqs_full, dqs_free
+  static constexpr int NBAR = 1 + 2 * NSQ + 2 + 8 + 2 + 2;
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
   static constexpr int SMEM_USED = MISC_OFF + 64;
   static constexpr int SMEM_ALLOC =
@@ -63,7 +67,6 @@ struct BwdParams {
   const float* lse;     // [BH][n]
   const float* delta;   // [BH][n]
   const float2* tab;    // [n][d/2] (cos, sin) of the RoPE angles
-  float* dQt;           // [BH][n][d] gradient w.r.t. Q~, accumulated (must start at zero)
   __nv_bfloat16* dK;    // [BH][n][d] rot^-1(dK~), bf16
   __nv_bfloat16* dV;    // [BH][n][d] bf16
   int n, BH, nk, causal;
@@ -72,15 +75,11 @@ struct BwdParams {
   unsigned long long limit_ns;
 };
 
-__device__ __forceinline__ void red_add_f32(float* addr, float v) {
-  asm volatile("red.global.add.f32 [%0], %1;" ::"l"(addr), "f"(v) : "memory");
-}
-
 template <int D>
 __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
 attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_l,
-                   const BwdParams p) {
+                   const __grid_constant__ CUtensorMap tm_dq, const BwdParams p) {
   using C = BwdCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -88,8 +87,7 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
   const uint32_t sbase = smem_u32(smem);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
   uint32_t* tslot = reinterpret_cast<uint32_t*>(smem + C::MISC_OFF);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::MISC_OFF + 4);
-  float2* ld_s = reinterpret_cast<float2*>(smem + C::LD_OFF);
+  const uint32_t abort_flag = smem_u32(smem + C::MISC_OFF + 4);
 
   const uint32_t b_kv = smem_u32(&bars[0]);
   auto b_qfull = [&](int s) { return smem_u32(&bars[1 + s]); };
@@ -102,6 +100,8 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
   auto b_dqfree = [&](int b) { return smem_u32(&bars[9 + 2 * C::NSQ + b]); };
   const uint32_t b_acc = smem_u32(&bars[11 + 2 * C::NSQ]);
   const uint32_t b_drain = smem_u32(&bars[12 + 2 * C::NSQ]);
+  const uint32_t b_dqsfull = smem_u32(&bars[13 + 2 * C::NSQ]);
+  const uint32_t b_dqsfree = smem_u32(&bars[14 + 2 * C::NSQ]);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   // head-major order: the key tiles of one (b, h) run side by side and share its Q~, l and
@@ -130,7 +130,9 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     }
     mbar_init(b_acc, 1);
     mbar_init(b_drain, 1);
-    *abort_flag = 0;
+    mbar_init(b_dqsfull, 128);
+    mbar_init(b_dqsfree, 1);
+    abort_set(abort_flag, 0);
     fence_barrier_init();
   }
   if (warp == 9) {
@@ -149,6 +151,7 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       tma_prefetch(&tm_k);
       tma_prefetch(&tm_v);
       tma_prefetch(&tm_l);
+      tma_prefetch(&tm_dq);
       mbar_expect_tx(b_kv, 2 * C::KTILE);
       for (int b = 0; b < C::KB; ++b) {
         tma_load_3d(sbase + C::K_OFF + b * C::KBLK, &tm_k, b_kv, 64 * b, kt * C::BK, bh);
@@ -173,15 +176,15 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
 #pragma unroll
       for (int h = 0; h < C::BQ / 32; ++h) {
         const int c = lane + 32 * h, q = q0 + c;
-        ld_s[s * C::BQ + c] = q < n ? make_float2(p.lse[(size_t)bh * n + q] * kLog2e,
-                                                  p.delta[(size_t)bh * n + q])
-                                    : make_float2(0.f, 0.f);
+        const float lz = q < n ? p.lse[(size_t)bh * n + q] * kLog2e : 0.f;
+        const float dz = q < n ? p.delta[(size_t)bh * n + q] : 0.f;
+        st_shared_v2f(sbase + C::LD_OFF + (s * C::BQ + c) * 8, lz, dz);
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(b_qfull(s));
       last = ii;
     }
-    if (lane == 0 && *abort_flag) {
+    if (lane == 0 && abort_get(abort_flag)) {
       mbar_drain(b_kv, 0, lim);
       for (int ii = (last - C::NSQ + 1 > 0 ? last - C::NSQ + 1 : 0); ii <= last; ++ii)
         mbar_drain(b_qfull(ii % C::NSQ), (ii / C::NSQ) & 1, lim);
@@ -283,7 +286,7 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       if (!(ok = mbar_wait_warp(b_pgfree(pb), ((ii >> 1) & 1) ^ 1, abort_flag, lim))) break;
       const uint32_t prow = sbase + C::P_OFF + pb * C::PG;
       const uint32_t grow = sbase + C::G_OFF + pb * C::PG;
-      const float4* ld4 = reinterpret_cast<const float4*>(ld_s + stg * C::BQ);
+      const uint32_t ld_row = sbase + C::LD_OFF + stg * C::BQ * 8;
       const bool full = key < n && q0 + C::BQ <= n && (!p.causal || key <= q0);
 #pragma unroll
       for (int c8 = 0; c8 < 8; ++c8) {
@@ -291,7 +294,8 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
 #pragma unroll
         for (int h = 0; h < 4; ++h) {
           const int c = c8 * 8 + h * 2;
-          const float4 lz = ld4[c >> 1];  // (lse_c, delta_c, lse_c+1, delta_c+1)
+          // (lse_c, delta_c, lse_c+1, delta_c+1)
+          const float4 lz = ld_shared_v4f(ld_row + (c >> 1) * 16);
           const int q = q0 + c;
           const bool v0 = full || (key < n && q < n && (!p.causal || key <= q));
           const bool v1 = full || (key < n && q + 1 < n && (!p.causal || key <= q + 1));
@@ -348,6 +352,8 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     // M = 64 puts row r in lane (r % 16) + 32 (r / 16)
     const int drow = (D == 128) ? (wq * 32 + lane) : (wq * 16 + lane);
     const bool has_row = (D == 128) || lane < 16;
+    const uint32_t stage = sbase + C::DQS_OFF;
+    const bool issuer = tid == 128;
     for (int ii = 0; ii < NI; ++ii) {
       const int pb = ii & 1;
       if (!mbar_wait_warp(b_dqfull(pb), (ii >> 1) & 1, abort_flag, lim)) break;
@@ -359,18 +365,31 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       tmem_wait_ld();
       tc_fence_before();
       mbar_arrive(b_dqfree(pb));
+      // the staging tile is free once the previous bulk reduction has read it
+      if (!mbar_wait_warp(b_dqsfree, (ii & 1) ^ 1, abort_flag, lim)) break;
       if (has_row) {
-        const int q0 = (i_start + ii) * C::BQ;
-        float* base = p.dQt + ((size_t)bh * n + q0) * D + drow;
-        const int qn = min(C::BQ, n - q0);
+        // row-major [q][d] fp32: for one q the lanes write consecutive d
 #pragma unroll
-        for (int c = 0; c < 32; ++c)
-          if (c < qn) red_add_f32(base + (size_t)c * D, __uint_as_float(r0[c]) * p.scale);
-#pragma unroll
-        for (int c = 0; c < 32; ++c)
-          if (32 + c < qn) red_add_f32(base + (size_t)(32 + c) * D, __uint_as_float(r1[c]) * p.scale);
+        for (int c = 0; c < 32; ++c) {
+          st_shared_f32(stage + (c * D + drow) * 4, __uint_as_float(r0[c]) * p.scale);
+          st_shared_f32(stage + ((32 + c) * D + drow) * 4, __uint_as_float(r1[c]) * p.scale);
+        }
       }
+      fence_proxy_async_smem();
+      mbar_arrive(b_dqsfull);
+      bool iok = true;
+      if (issuer) {
+        iok = mbar_wait(b_dqsfull, ii & 1, abort_flag, lim);
+        if (iok) {
+          tma_reduce_add_3d(&tm_dq, stage, 0, (i_start + ii) * C::BQ, bh);
+          bulk_commit();
+          bulk_wait_read0();
+          mbar_arrive(b_dqsfree);
+        }
+      }
+      if (!__all_sync(0xffffffffu, iok)) break;  // leave the loop together
     }
+    if (issuer) bulk_wait0();  // the reductions have landed before the CTA leaves
   }
   tc_fence_before();
   __syncthreads();

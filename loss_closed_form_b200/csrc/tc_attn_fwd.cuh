@@ -71,7 +71,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
   const uint32_t sbase = smem_u32(smem);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
   uint32_t* tslot = reinterpret_cast<uint32_t*>(smem + C::MISC_OFF);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::MISC_OFF + 4);
+  const uint32_t abort_flag = smem_u32(smem + C::MISC_OFF + 4);
   float* red = reinterpret_cast<float*>(smem + C::MISC_OFF + 16);  // 4 partial sums
 
   const uint32_t b_q = smem_u32(&bars[0]);
@@ -107,7 +107,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
       mbar_init(b_pvdone(b), 1);
     }
     mbar_init(b_drain, 1);
-    *abort_flag = 0;
+    abort_set(abort_flag, 0);
     fence_barrier_init();
   }
   if (warp == 5) {
@@ -145,7 +145,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                       j * C::BN, bh);
         last_v = j;
       }
-      if (*abort_flag) {
+      if (abort_get(abort_flag)) {
         // let the copies already issued land before the CTA leaves (at most one pending
         // phase per stage: a stage is refilled only after its previous contents were used)
         mbar_drain(b_q, 0, lim);
@@ -259,29 +259,24 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
           tmem_wait_st();
         }
       }
-      float psum = 0.f;
-      uint32_t pk[64];
-#pragma unroll
-      for (int i = 0; i < 64; ++i) {
-        const float p0 = ex2(x[2 * i] - m), p1 = ex2(x[2 * i + 1] - m);
-        psum += p0 + p1;
-        pk[i] = pack_bf16x2(p0, p1);
-      }
-      l += psum;
       if (j >= 2) {  // P buffer sb was read by the product of tile j - 2
         if (!(ok = mbar_wait_warp(b_pvdone(sb), ((j - 2) >> 1) & 1, abort_flag, lim))) break;
         tc_fence_after();
       }
       const uint32_t p_addr = tmem + lane_base + (sb ? C::T_P1 : C::T_P0);
-      {
-        uint32_t r[32];
+      float psum = 0.f;
 #pragma unroll
-        for (int i = 0; i < 32; ++i) r[i] = pk[i];
-        tmem_st32(p_addr, r);
+      for (int h = 0; h < 2; ++h) {
+        uint32_t pk[32];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) r[i] = pk[32 + i];
-        tmem_st32(p_addr + 32, r);
+        for (int i = 0; i < 32; ++i) {
+          const float p0 = ex2(x[64 * h + 2 * i] - m), p1 = ex2(x[64 * h + 2 * i + 1] - m);
+          psum += p0 + p1;
+          pk[i] = pack_bf16x2(p0, p1);
+        }
+        tmem_st32(p_addr + 32 * h, pk);
       }
+      l += psum;
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(b_pfull(sb));

@@ -56,7 +56,7 @@ proj_rope_tc_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_cons
   const uint32_t sbase = smem_u32(smem);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
   uint32_t* tslot = reinterpret_cast<uint32_t*>(smem + C::MISC_OFF);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::MISC_OFF + 4);
+  const uint32_t abort_flag = smem_u32(smem + C::MISC_OFF + 4);
   const uint32_t b_full = smem_u32(&bars[0]), b_mma = smem_u32(&bars[1]);
   const int tid = threadIdx.x, warp = tid >> 5;
   const int bh = blockIdx.x, rt = blockIdx.y, z = blockIdx.z, h = bh % p.H;
@@ -66,7 +66,7 @@ proj_rope_tc_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_cons
   if (tid == 0) {
     mbar_init(b_full, 1);
     mbar_init(b_mma, 1);
-    *abort_flag = 0;
+    abort_set(abort_flag, 0);
     fence_barrier_init();
   }
   if (warp == 0) {
@@ -97,7 +97,7 @@ proj_rope_tc_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_cons
     if (!ok) mbar_drain(b_full, 0, lim);
   }
   __syncwarp();
-  ok = mbar_wait_warp(b_mma, 0, abort_flag, lim) && !*abort_flag;
+  ok = mbar_wait_warp(b_mma, 0, abort_flag, lim) && !abort_get(abort_flag);
   tc_fence_after();
   if (ok) {
     const int row = rt * C::BM + tid;
@@ -191,7 +191,7 @@ dw_tc_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_constant__ 
   const uint32_t sbase = smem_u32(smem);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
   uint32_t* tslot = reinterpret_cast<uint32_t*>(smem + C::MISC_OFF);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::MISC_OFF + 4);
+  const uint32_t abort_flag = smem_u32(smem + C::MISC_OFF + 4);
   auto b_full = [&](int s) { return smem_u32(&bars[s]); };
   auto b_empty = [&](int s) { return smem_u32(&bars[C::NS + s]); };
   const uint32_t b_done = smem_u32(&bars[2 * C::NS]);
@@ -211,7 +211,7 @@ dw_tc_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_constant__ 
     }
     mbar_init(b_done, 1);
     mbar_init(b_drain, 1);
-    *abort_flag = 0;
+    abort_set(abort_flag, 0);
     fence_barrier_init();
   }
   if (warp == 5) {
@@ -238,7 +238,7 @@ dw_tc_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_constant__ 
         }
         last = t;
       }
-      if (*abort_flag)
+      if (abort_get(abort_flag))
         for (int t = (last - C::NS + 1 > 0 ? last - C::NS + 1 : 0); t <= last; ++t)
           mbar_drain(b_full(t % C::NS), (t / C::NS) & 1, lim);
     }

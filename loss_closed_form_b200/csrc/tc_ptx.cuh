@@ -47,19 +47,30 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// The CTA's abort flag lives in shared memory and is read / written with explicit
+// shared-space accesses (a generic pointer would send every poll through L1TEX).
+__device__ __forceinline__ int abort_get(uint32_t flag) {
+  int v;
+  asm volatile("ld.volatile.shared.s32 %0, [%1];" : "=r"(v) : "r"(flag) : "memory");
+  return v;
+}
+__device__ __forceinline__ void abort_set(uint32_t flag, int v) {
+  asm volatile("st.volatile.shared.s32 [%0], %1;" ::"r"(flag), "r"(v) : "memory");
+}
+
 // Wait for the phase with parity `parity` of barrier `bar` to complete.  Gives up when the
-// CTA's abort flag is set, or after `limit_ns` of global time: then records a timeout in
-// the library status word, sets the abort flag and returns false.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+// CTA's abort flag (shared address `abort_flag`) is set, or after `limit_ns` of global time:
+// then records a timeout in the library status word, sets the abort flag and returns false.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint32_t abort_flag,
                                           uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
-    if (*abort_flag) return false;
+    if (abort_get(abort_flag)) return false;
     if (globaltimer() - t0 > limit_ns) {
       flag_error(kDevTimeout);
-      *abort_flag = 1;
+      abort_set(abort_flag, 1);
       return false;
     }
   }
@@ -67,8 +78,8 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
 
 // Warp-uniform form: every lane of the calling warp must call it; true only if the wait
 // succeeded for all lanes (so .sync.aligned TMEM instructions that follow stay convergent).
-__device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity,
-                                               volatile int* abort_flag, uint64_t limit_ns) {
+__device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity, uint32_t abort_flag,
+                                               uint64_t limit_ns) {
   const bool ok = mbar_wait(bar, parity, abort_flag, limit_ns);
   return __all_sync(0xffffffffu, ok);
 }
@@ -247,6 +258,45 @@ __device__ __forceinline__ float ex2(float x) {
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);  // .x = lo (low 16 bits), .y = hi
   return *reinterpret_cast<uint32_t*>(&v);
+}
+
+__device__ __forceinline__ float4 ld_shared_v4f(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(addr));
+  return v;
+}
+__device__ __forceinline__ void st_shared_f32(uint32_t addr, float v) {
+  asm volatile("st.shared.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
+}
+__device__ __forceinline__ void st_shared_v2f(uint32_t addr, float a, float b) {
+  asm volatile("st.shared.v2.f32 [%0], {%1, %2};" ::"r"(addr), "f"(a), "f"(b) : "memory");
+}
+__device__ __forceinline__ void st_shared_s32(uint32_t addr, int v) {
+  asm volatile("st.shared.s32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+
+// TMA bulk reduce-add of an fp32 tile from shared memory into global memory (3-D map); the
+// coordinates must be non-negative, rows past the map's extent are skipped.
+__device__ __forceinline__ void tma_reduce_add_3d(const CUtensorMap* map, uint32_t src, int x,
+                                                  int y, int z) {
+  asm volatile(
+      "cp.reduce.async.bulk.tensor.3d.global.shared::cta.add.tile.bulk_group"
+      " [%0, {%2, %3, %4}], [%1];" ::"l"(reinterpret_cast<uint64_t>(map)),
+      "r"(src), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
+__device__ __forceinline__ void bulk_commit() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// Wait until the shared-memory source of every committed bulk group has been read.
+__device__ __forceinline__ void bulk_wait_read0() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+// Wait until every committed bulk group has completed.
+__device__ __forceinline__ void bulk_wait0() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
 
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,

@@ -30,7 +30,7 @@ probe_mma_kernel(const __nv_bfloat16* __restrict__ A, const __nv_bfloat16* __res
   uint8_t* sB = smem + kSmemA;
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + kSmemA + kSmemB);
   uint32_t* tslot = reinterpret_cast<uint32_t*>(bar + 1);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(tslot + 1);
+  const uint32_t abort_flag = smem_u32(tslot + 1);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
   // A into swizzled smem: 16-byte chunks of 8 consecutive elements along the major axis
@@ -72,7 +72,7 @@ probe_mma_kernel(const __nv_bfloat16* __restrict__ A, const __nv_bfloat16* __res
   }
   if (tid == 0) {
     mbar_init(smem_u32(bar), 1);
-    *abort_flag = 0;
+    abort_set(abort_flag, 0);
     fence_barrier_init();
   }
   fence_proxy_async_smem();
@@ -145,15 +145,16 @@ probe_mma_kernel(const __nv_bfloat16* __restrict__ A, const __nv_bfloat16* __res
 
 __global__ void probe_timeout_kernel(unsigned long long limit_ns, int* waited_ok) {
   __shared__ __align__(8) uint64_t bar;
-  __shared__ int abort_flag;
+  __shared__ int abort_word;
+  const uint32_t abort_flag = smem_u32(&abort_word);
   if (threadIdx.x == 0) {
     mbar_init(smem_u32(&bar), 1);
-    abort_flag = 0;
+    abort_set(abort_flag, 0);
     fence_barrier_init();
   }
   __syncthreads();
   // nothing ever arrives on `bar`: the wait must give up after limit_ns
-  const bool ok = mbar_wait(smem_u32(&bar), 0, &abort_flag, limit_ns);
+  const bool ok = mbar_wait(smem_u32(&bar), 0, abort_flag, limit_ns);
   if (threadIdx.x == 0) *waited_ok = ok ? 1 : 0;
 }
 
