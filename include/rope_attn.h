@@ -142,6 +142,38 @@ int32_t rope_attn_profile_read(float* ms, int32_t* launches, int32_t max_kernels
 /* Static name of kernel id `id` (NULL if out of range). */
 const char* rope_attn_kernel_name(int32_t id);
 
+/*
+ * Size of the scratch array behind rope_attn_step_noalloc: a file-scope device array of the
+ * library that every GPU which loads the library holds until the process exits.
+ */
+#define RA_NOALLOC_SCRATCH_BYTES (16u * 1024u * 1024u)
+
+/*
+ * One whole step (rope_attn_fwd with the loss, then rope_attn_loss_bwd reusing the forward's
+ * intermediates) for callers that cannot call cudaMalloc, for example code that may not take
+ * the device-wide synchronisation an allocation can cause, or that runs inside a component
+ * whose device memory is owned by someone else.  There is no counterpart of this entry point
+ * in the paper; it exists only for such callers.
+ *
+ * The caller passes inputs (p, with E) and outputs exactly as for rope_attn_fwd and
+ * rope_attn_loss_bwd: O, lse, loss (may be NULL), dWQ, dWK, dWV.  Instead of a caller-owned
+ * workspace the step uses the library's static scratch array of RA_NOALLOC_SCRATCH_BYTES on
+ * the current device.  Nothing is allocated or freed: no cudaMalloc, cudaFree or allocating
+ * library routine is called.
+ *
+ * Limits and behaviour:
+ *   - a problem whose workspace (rope_attn_workspace_bytes) exceeds RA_NOALLOC_SCRATCH_BYTES is
+ *     rejected with RA_ERR_WORKSPACE before anything is launched;
+ *   - the first call on a device looks up the scratch array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call before any stream
+ *     capture;
+ *   - every call on a device shares the one scratch array, which keeps the last call's contents;
+ *     the step clears what must start at zero itself, but calls whose work overlaps on the GPU
+ *     (different streams, or different host threads) race on the scratch: order them.
+ */
+ra_status rope_attn_step_noalloc(const ra_problem* p, void* O, float* lse, float* loss,
+                                 float* dWQ, float* dWK, float* dWV, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

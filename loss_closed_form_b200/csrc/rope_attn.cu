@@ -8,6 +8,7 @@
 #include <stdint.h>
 #include <string.h>
 
+#include <mutex>
 #include <vector>
 
 #include <cudaTypedefs.h>
@@ -566,6 +567,32 @@ ra_status tc_bwd(const ra_problem* p, const void* O, const float* lse, float* lo
   return launch_status();
 }
 
+// ---------------------------------------------------------------------------------------
+// Scratch for rope_attn_step_noalloc: lives in the library's device image, so every GPU that
+// loads the library holds it until exit.  Host code must not use the symbol's name as a device
+// address (it names a host-side shadow); the device address comes from cudaGetSymbolAddress.
+// ---------------------------------------------------------------------------------------
+static __device__ __align__(256) unsigned char g_noalloc_scratch[RA_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mutex;
+void* g_noalloc_addr[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device (looked up once per device).
+ra_status noalloc_scratch(void** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return RA_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return RA_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (!g_noalloc_addr[dev]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr) return RA_ERR_CUDA;
+    g_noalloc_addr[dev] = ptr;
+  }
+  *out = g_noalloc_addr[dev];
+  return RA_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -606,6 +633,32 @@ ra_status rope_attn_loss_bwd(const ra_problem* p, const void* O, const float* ls
   if (p->dtype == RA_F32)
     return simt_bwd(p, O, lse, loss, dWQ, dWK, dWV, ws, ws_holds_fwd, st);
   return tc_bwd(p, O, lse, loss, dWQ, dWK, dWV, ws, ws_holds_fwd, st);
+}
+
+ra_status rope_attn_step_noalloc(const ra_problem* p, void* O, float* lse, float* loss,
+                                 float* dWQ, float* dWK, float* dWV, void* stream) {
+  ra_status s = check_problem(p);
+  if (s != RA_OK) return s;
+  if (!p->E || !O || !lse || !dWQ || !dWK || !dWV) return RA_ERR_INVALID_ARG;
+  if (!is_aligned(O, 16) || !is_aligned(lse, 4) || (loss && !is_aligned(loss, 4)) ||
+      !is_aligned(dWQ, 16) || !is_aligned(dWK, 16) || !is_aligned(dWV, 16))
+    return RA_ERR_ALIGNMENT;
+  const size_t need = make_layout(p).total;
+  if (need > RA_NOALLOC_SCRATCH_BYTES) return RA_ERR_WORKSPACE;
+  void* ws = nullptr;
+  s = noalloc_scratch(&ws);
+  if (s != RA_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // the forward writes every intermediate the backward reads; the backward zeroes its dQ~
+  // accumulator itself, so no state of an earlier call leaks into this one
+  if (p->dtype == RA_F32) {
+    s = simt_fwd<float>(p, O, lse, loss, ws, st);
+    if (s != RA_OK) return s;
+    return simt_bwd(p, O, lse, loss, dWQ, dWK, dWV, ws, 1, st);
+  }
+  s = tc_fwd(p, O, lse, loss, ws, st);
+  if (s != RA_OK) return s;
+  return tc_bwd(p, O, lse, loss, dWQ, dWK, dWV, ws, 1, st);
 }
 
 ra_status rope_attn_last_error(void* stream) {

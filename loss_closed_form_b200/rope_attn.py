@@ -20,7 +20,11 @@ RA_F32, RA_BF16 = 0, 1
 # Every symbol include/rope_attn.h declares.
 EXPORTED = ("rope_attn_workspace_bytes", "rope_attn_fwd", "rope_attn_loss_bwd",
             "rope_attn_last_error", "rope_attn_status_string", "rope_attn_launch_count",
-            "rope_attn_profile_enable", "rope_attn_profile_read", "rope_attn_kernel_name")
+            "rope_attn_profile_enable", "rope_attn_profile_read", "rope_attn_kernel_name",
+            "rope_attn_step_noalloc")
+
+# Capacity of the static scratch behind rope_attn_step_noalloc (RA_NOALLOC_SCRATCH_BYTES).
+NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
 
 
 class Problem(ctypes.Structure):
@@ -73,6 +77,8 @@ def load() -> ctypes.CDLL:
     lib.rope_attn_profile_read.restype = i32
     lib.rope_attn_kernel_name.argtypes = [i32]
     lib.rope_attn_kernel_name.restype = ctypes.c_char_p
+    lib.rope_attn_step_noalloc.argtypes = [P, vp, vp, vp, vp, vp, vp, vp]
+    lib.rope_attn_step_noalloc.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -142,6 +148,18 @@ def loss_bwd(prob: Problem, O, lse, loss, dWQ, dWK, dWV, ws, ws_holds_fwd=False,
                                    _stream(stream))
     if st != RA_OK:
         raise RopeAttnError(st, "rope_attn_loss_bwd")
+
+
+def step_noalloc(prob: Problem, O, lse, loss, dWQ, dWK, dWV, stream=None) -> None:
+    """rope_attn_step_noalloc: forward + backward on the library's static scratch.
+
+    For callers that cannot allocate device memory; problems whose workspace exceeds
+    NOALLOC_SCRATCH_BYTES raise RopeAttnError(RA_ERR_WORKSPACE).
+    """
+    st = load().rope_attn_step_noalloc(ctypes.byref(prob), _ptr(O), _ptr(lse), _ptr(loss),
+                                       _ptr(dWQ), _ptr(dWK), _ptr(dWV), _stream(stream))
+    if st != RA_OK:
+        raise RopeAttnError(st, "rope_attn_step_noalloc")
 
 
 def last_error(stream=None) -> int:
