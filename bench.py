@@ -71,6 +71,25 @@ def workload_config(w, n_gpus):
 
 
 # ---------------------------------------------------------------------------------------
+# multi-rank aggregation (host logic; exercised on CPU with gloo in the tests)
+# ---------------------------------------------------------------------------------------
+def max_over_ranks(ms: float, world: int, device=None) -> float:
+    """Slowest rank's time: every rank contributes its own device-timed milliseconds."""
+    if world <= 1:
+        return ms
+    import torch
+    import torch.distributed as dist
+    x = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(x, op=dist.ReduceOp.MAX)
+    return float(x.item())
+
+
+def whole_job_tflops(flops_per_rank_step: float, steps: int, world: int, ms_max: float) -> float:
+    """Work of all ranks (weak scaling: each rank runs its own copy) over the slowest time."""
+    return world * flops_per_rank_step * steps / (ms_max * 1e-3) / 1e12
+
+
+# ---------------------------------------------------------------------------------------
 # clocks sampled with nvidia-smi during the timed region
 # ---------------------------------------------------------------------------------------
 class ClockSampler:
@@ -194,11 +213,7 @@ def run_ours(args, rank, world, local_rank):
     st = ra.last_error()
     if st != ra.RA_OK:
         raise RuntimeError(f"kernel status after timing: {ra.status_string(st)}")
-    ms_max = ms
-    if world > 1:
-        x = torch.tensor([ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(x, op=dist.ReduceOp.MAX)
-        ms_max = float(x.item())
+    ms_max = max_over_ranks(ms, world, dev)
 
     # ---- end to end: pinned host inputs -> device, step, loss + dW back to the host -----
     e2e = None
@@ -229,14 +244,10 @@ def run_ours(args, rank, world, local_rank):
         e1.record(stream)
         torch.cuda.synchronize(dev)
         barrier()
-        ms_e2e = e0.elapsed_time(e1)
-        if world > 1:
-            x = torch.tensor([ms_e2e], dtype=torch.float64, device=dev)
-            dist.all_reduce(x, op=dist.ReduceOp.MAX)
-            ms_e2e = float(x.item())
+        ms_e2e = max_over_ranks(e0.elapsed_time(e1), world, dev)
         if not math.isfinite(float(out_host["loss"])):
             raise RuntimeError("non-finite loss in the end-to-end run")
-        e2e = {"value": round(world * flops * args.steps / (ms_e2e * 1e-3) / 1e12, 3),
+        e2e = {"value": round(whole_job_tflops(flops, args.steps, world, ms_e2e), 3),
                "unit": "TFLOP/s", "ms_per_step": round(ms_e2e / args.steps, 4),
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
 
@@ -249,7 +260,7 @@ def run_ours(args, rank, world, local_rank):
     top_name, (top_ms, top_n) = top
     avg_ms = top_ms / max(1, top_n)
     roof = roofline(w, top_name, avg_ms, pk, src)
-    value = world * flops * args.steps / (ms_max * 1e-3) / 1e12
+    value = whole_job_tflops(flops, args.steps, world, ms_max)
     total_kernel_ms = sum(v[0] for v in per_kernel.values())
     line = {
         "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world,
