@@ -290,7 +290,7 @@ def roofline(w, kname, avg_ms, pk, src):
     tensor_kernels = {"attn_bwd_tc": 10.0 * d * P * BH, "attn_fwd_tc": 4.0 * d * P * BH}
     simt_kernels = {"attn_bwd_simt": 10.0 * d * P * BH, "attn_fwd_simt": 4.0 * d * P * BH,
                     "proj_rope_simt": 6.0 * n * d * d * BH, "dw_partial_simt": 6.0 * n * d * d * BH}
-    traffic = measured_traffic(kname)
+    traffic = measured_traffic(kname) if w.name == DEFAULT_WORKLOAD else None
     if kname in tensor_kernels:
         flop = tensor_kernels[kname]
         peak = pk["bf16_tflops"]
@@ -313,8 +313,29 @@ def roofline(w, kname, avg_ms, pk, src):
             "unit": "GB/s", "frac": None, "traffic": traffic, "avg_launch_ms": round(avg_ms, 4)}
 
 
+# source files that define each tensor-core kernel; a committed traffic figure counts only
+# while these files are unchanged since its ncu capture
+KERNEL_SOURCES = {
+    "attn_bwd_tc": ("tc_attn_bwd.cuh", "tc_ptx.cuh", "common.cuh"),
+    "attn_fwd_tc": ("tc_attn_fwd.cuh", "tc_ptx.cuh", "common.cuh"),
+}
+
+
+def kernel_source_sha(kname):
+    import hashlib
+    files = KERNEL_SOURCES.get(kname)
+    if not files:
+        return None
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "loss_closed_form_b200", "csrc")
+    for f in files:
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
 def measured_traffic(kname):
-    """DRAM bytes per launch from a committed ncu summary, if it matches the current source."""
+    """DRAM bytes per launch from profiles/traffic.json, if it matches the current source."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
@@ -322,22 +343,11 @@ def measured_traffic(kname):
     except (OSError, ValueError):
         return None
     ent = rec.get(kname)
-    if not ent:
+    if not ent or ent.get("workload") is None:
         return None
-    if ent.get("source_sha") != kernel_source_sha():
+    if ent.get("source_sha") != kernel_source_sha(kname):
         return None
     return ent.get("dram_bytes_per_launch")
-
-
-def kernel_source_sha():
-    import hashlib
-    h = hashlib.sha256()
-    csrc = os.path.join(ROOT, "loss_closed_form_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
-        if f.endswith((".cu", ".cuh")):
-            with open(os.path.join(csrc, f), "rb") as fh:
-                h.update(fh.read())
-    return h.hexdigest()[:16]
 
 
 # ---------------------------------------------------------------------------------------
