@@ -16,10 +16,11 @@
 // Definitions: "RoPE Attention kan bijna lineair worden getraind", Methodologie 1 (s, l,
 // beta, gamma) and 2 (gamma_1 = diag(s) beta, gamma_2 = s s^T beta).
 //
-// Warp roles (320 threads): warps 0-3 softmax / gamma and the dK, dV epilogue (one key row
-// per thread), warps 4-7 drain dQ~ from TMEM into the staging tile (thread 128 issues the
-// bulk reduction), warp 8 TMA producer (it also stages the query tile's lse and delta),
-// warp 9 MMA issuer and TMEM owner.
+// Warp roles (448 threads): warps 0-7 softmax / gamma (two warpgroups over the same 128 key
+// rows, each taking half of the 64 query columns) and the epilogue (warps 0-3 dK, 4-7 dV),
+// warps 8-11 drain dQ~ from TMEM into the staging tile (thread 256 issues the bulk
+// reduction), warp 12 TMA producer (it also stages the query tile's lse and delta), warp 13
+// MMA issuer and TMEM owner.
 #pragma once
 #include "tc_ptx.cuh"
 
@@ -55,7 +56,8 @@ struct BwdCfg {
   static constexpr int SMEM_USED = MISC_OFF + 64;
   static constexpr int SMEM_ALLOC =
       (SMEM_USED + 1024 > 120 * 1024) ? SMEM_USED + 1024 : 120 * 1024;
-  static constexpr int THREADS = 320;
+  static constexpr int THREADS = 448;
+  static constexpr int W_DRAIN = 8, W_PROD = 12, W_MMA = 13;
   // TMEM columns
   static constexpr uint32_t T_S = 0, T_B = 64, T_DQ0 = 128, T_DQ1 = 192, T_DK = 256,
                             T_DV = 256 + D;
@@ -121,9 +123,9 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       mbar_init(b_qempty(s), 1);
     }
     mbar_init(b_sfull, 1);
-    mbar_init(b_sfree, 128);
+    mbar_init(b_sfree, 256);
     for (int b = 0; b < 2; ++b) {
-      mbar_init(b_pgfull(b), 128);
+      mbar_init(b_pgfull(b), 256);
       mbar_init(b_pgfree(b), 1);
       mbar_init(b_dqfull(b), 1);
       mbar_init(b_dqfree(b), 128);
@@ -135,7 +137,7 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     abort_set(abort_flag, 0);
     fence_barrier_init();
   }
-  if (warp == 9) {
+  if (warp == C::W_MMA) {
     tmem_alloc(smem_u32(tslot), C::T_COLS);
     tmem_relinquish();
   }
@@ -144,7 +146,7 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
   tc_fence_after();
   const uint32_t tmem = *tslot;
 
-  if (warp == 8) {
+  if (warp == C::W_PROD) {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
       tma_prefetch(&tm_q);
@@ -189,7 +191,7 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       for (int ii = (last - C::NSQ + 1 > 0 ? last - C::NSQ + 1 : 0); ii <= last; ++ii)
         mbar_drain(b_qfull(ii % C::NSQ), (ii / C::NSQ) & 1, lim);
     }
-  } else if (warp == 9) {
+  } else if (warp == C::W_MMA) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc_sb = idesc_bf16_f32(128, C::BQ, false, false);
@@ -256,10 +258,13 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         mbar_drain(b_drain, 0, lim);
       }
     }
-  } else if (warp < 4) {
+  } else if (warp < C::W_DRAIN) {
     // ------------------------------------------------------------------ P^T, gamma^T
-    const int key = kt * C::BK + tid;
-    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    // warp w reaches TMEM lanes 32 (w % 4) ...; warpgroup `half` takes query columns
+    // 32 half .. 32 half + 31 of the 64
+    const int row = tid & 127, half = warp >> 2;
+    const int key = kt * C::BK + row;
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
     bool ok = true;
     for (int ii = 0; ii < NI; ++ii) {
       const int q0 = (i_start + ii) * C::BQ;
@@ -268,35 +273,28 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       if (!(ok = mbar_wait_warp(b_qfull(stg), (ii / C::NSQ) & 1, abort_flag, lim))) break;
       if (!(ok = mbar_wait_warp(b_sfull, ii & 1, abort_flag, lim))) break;
       tc_fence_after();
-      uint32_t sr[64], br[64];
-      {
-        uint32_t (&s0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[0]);
-        uint32_t (&s1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[32]);
-        uint32_t (&b0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&br[0]);
-        uint32_t (&b1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&br[32]);
-        tmem_ld32(tmem + lane_base + C::T_S, s0);
-        tmem_ld32(tmem + lane_base + C::T_S + 32, s1);
-        tmem_ld32(tmem + lane_base + C::T_B, b0);
-        tmem_ld32(tmem + lane_base + C::T_B + 32, b1);
-        tmem_wait_ld();
-      }
+      uint32_t sr[32], br[32];
+      tmem_ld32(tmem + lane_base + C::T_S + 32 * half, sr);
+      tmem_ld32(tmem + lane_base + C::T_B + 32 * half, br);
+      tmem_wait_ld();
       tc_fence_before();
       mbar_arrive(b_sfree);
       const int pb = ii & 1;
       if (!(ok = mbar_wait_warp(b_pgfree(pb), ((ii >> 1) & 1) ^ 1, abort_flag, lim))) break;
       const uint32_t prow = sbase + C::P_OFF + pb * C::PG;
       const uint32_t grow = sbase + C::G_OFF + pb * C::PG;
-      const uint32_t ld_row = sbase + C::LD_OFF + stg * C::BQ * 8;
-      const bool full = key < n && q0 + C::BQ <= n && (!p.causal || key <= q0);
+      const uint32_t ld_row = sbase + C::LD_OFF + (stg * C::BQ + 32 * half) * 8;
+      const int qh = q0 + 32 * half;
+      const bool full = key < n && qh + 32 <= n && (!p.causal || key <= qh);
 #pragma unroll
-      for (int c8 = 0; c8 < 8; ++c8) {
+      for (int c8 = 0; c8 < 4; ++c8) {
         uint32_t pw[4], gw[4];
 #pragma unroll
         for (int h = 0; h < 4; ++h) {
           const int c = c8 * 8 + h * 2;
           // (lse_c, delta_c, lse_c+1, delta_c+1)
           const float4 lz = ld_shared_v4f(ld_row + (c >> 1) * 16);
-          const int q = q0 + c;
+          const int q = qh + c;
           const bool v0 = full || (key < n && q < n && (!p.causal || key <= q));
           const bool v1 = full || (key < n && q + 1 < n && (!p.causal || key <= q + 1));
           const float p0 = v0 ? ex2(__uint_as_float(sr[c]) * p.scale_log2 - lz.x) : 0.f;
@@ -305,55 +303,56 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
           gw[h] = pack_bf16x2(p0 * (__uint_as_float(br[c]) - lz.y),
                               p1 * (__uint_as_float(br[c + 1]) - lz.w));
         }
-        const uint32_t off = sw128_offset(tid, c8);
+        const uint32_t off = sw128_offset(row, 4 * half + c8);
         st_shared_v4(prow + off, pw[0], pw[1], pw[2], pw[3]);
         st_shared_v4(grow + off, gw[0], gw[1], gw[2], gw[3]);
       }
       fence_proxy_async_smem();
       mbar_arrive(b_pgfull(pb));
     }
-    // ---- dK = rot^-1(scale * sum gamma^T Q~), dV = sum P^T l: one key row per thread
+    // ---- dK = rot^-1(scale * sum gamma^T Q~) (warps 0-3), dV = sum P^T l (warps 4-7):
+    //      one key row per thread
     if (ok) ok = mbar_wait_warp(b_acc, 0, abort_flag, lim);
     if (ok) {
       tc_fence_after();
       const size_t ro = ((size_t)bh * n + key) * D;
       const float2* tr = p.tab + (size_t)(key < n ? key : 0) * (D / 2);
+      __nv_bfloat16* dst = (half == 0 ? p.dK : p.dV) + ro;
+      const uint32_t src = tmem + lane_base + (half == 0 ? C::T_DK : C::T_DV);
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
-        uint32_t rk[32], rv[32];
-        tmem_ld32(tmem + lane_base + C::T_DK + 32 * c, rk);
-        tmem_ld32(tmem + lane_base + C::T_DV + 32 * c, rv);
+        uint32_t r[32];
+        tmem_ld32(src + 32 * c, r);
         tmem_wait_ld();
         if (key < n) {
-          uint32_t wk[16], wv[16];
+          uint32_t w[16];
 #pragma unroll
           for (int k = 0; k < 16; ++k) {
-            const float x0 = __uint_as_float(rk[2 * k]) * p.scale;
-            const float x1 = __uint_as_float(rk[2 * k + 1]) * p.scale;
-            const float2 cs = tr[16 * c + k];  // rotation by -phi
-            wk[k] = pack_bf16x2(x0 * cs.x + x1 * cs.y, -x0 * cs.y + x1 * cs.x);
-            wv[k] = pack_bf16x2(__uint_as_float(rv[2 * k]), __uint_as_float(rv[2 * k + 1]));
+            const float x0 = __uint_as_float(r[2 * k]), x1 = __uint_as_float(r[2 * k + 1]);
+            if (half == 0) {
+              const float y0 = x0 * p.scale, y1 = x1 * p.scale;
+              const float2 cs = tr[16 * c + k];  // rotation by -phi
+              w[k] = pack_bf16x2(y0 * cs.x + y1 * cs.y, -y0 * cs.y + y1 * cs.x);
+            } else {
+              w[k] = pack_bf16x2(x0, x1);
+            }
           }
-          uint4* dk = reinterpret_cast<uint4*>(p.dK + ro + 32 * c);
-          uint4* dv = reinterpret_cast<uint4*>(p.dV + ro + 32 * c);
+          uint4* o = reinterpret_cast<uint4*>(dst + 32 * c);
 #pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            dk[v] = make_uint4(wk[4 * v], wk[4 * v + 1], wk[4 * v + 2], wk[4 * v + 3]);
-            dv[v] = make_uint4(wv[4 * v], wv[4 * v + 1], wv[4 * v + 2], wv[4 * v + 3]);
-          }
+          for (int v = 0; v < 4; ++v) o[v] = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
         }
       }
     }
   } else {
-    // ------------------------------------------------------------------ dQ~ drain (warps 4-7)
-    const int wq = warp - 4;
+    // ------------------------------------------------------------------ dQ~ drain (warps 8-11)
+    const int wq = warp - C::W_DRAIN;
     const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
     // accumulator row (head-dimension index) held by this lane: M = 128 puts row r in lane r,
     // M = 64 puts row r in lane (r % 16) + 32 (r / 16)
     const int drow = (D == 128) ? (wq * 32 + lane) : (wq * 16 + lane);
     const bool has_row = (D == 128) || lane < 16;
     const uint32_t stage = sbase + C::DQS_OFF;
-    const bool issuer = tid == 128;
+    const bool issuer = tid == 32 * C::W_DRAIN;
     for (int ii = 0; ii < NI; ++ii) {
       const int pb = ii & 1;
       if (!mbar_wait_warp(b_dqfull(pb), (ii >> 1) & 1, abort_flag, lim)) break;
@@ -393,7 +392,7 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == C::W_MMA) {
     tc_fence_after();
     tmem_dealloc(tmem, C::T_COLS);
   }
