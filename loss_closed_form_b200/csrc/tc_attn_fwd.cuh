@@ -13,8 +13,10 @@
 // 2^8 (log2 units): O and l keep one common reference, so the final O / l is unchanged and
 // P stays <= 256 in bf16.
 //
-// Warp roles (192 threads): warps 0-3 softmax + epilogue, warp 4 TMA producer, warp 5 MMA
-// issuer and TMEM owner.
+// Warp roles (320 threads): warps 0-7 softmax + epilogue (two warpgroups over the same 128
+// query rows, each taking 64 of the 128 key columns of a tile; the row maximum, row sum and
+// <l, O> are combined through shared memory), warp 8 TMA producer, warp 9 MMA issuer and
+// TMEM owner.
 #pragma once
 #include "tc_ptx.cuh"
 
@@ -34,14 +36,18 @@ struct FwdCfg {
   static constexpr int V_OFF = K_OFF + NS * TILE;
   static constexpr int BAR_OFF = V_OFF + NS * TILE;
   // barriers: q_full, k_full[NS], k_empty[NS], v_full[NS], v_empty[NS], s_full[2],
-  //           p_full[2], pv_done[2], drain
-  static constexpr int NBAR = 1 + 4 * NS + 6 + 1;
-  static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;  // tmem slot, abort flag, reduction
-  static constexpr int SMEM_USED = MISC_OFF + 64;
+  //           p_full[2], pv_done[2], drain, xch[2], ep1, ep2
+  static constexpr int NBAR = 1 + 4 * NS + 6 + 1 + 4;
+  static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;  // tmem slot, abort flag, 8 partial sums
+  static constexpr int XCH_OFF = MISC_OFF + 64;        // float [2 buffers][2 halves][128 rows]
+  static constexpr int EPL_OFF = XCH_OFF + 2 * 2 * 128 * 4;  // float [2 halves][128]: row sums
+  static constexpr int EPD_OFF = EPL_OFF + 2 * 128 * 4;      // float [128]: <l, O> of half 1
+  static constexpr int SMEM_USED = EPD_OFF + 128 * 4;
   // at least half of the SM's shared memory: one CTA per SM, so the 512-column TMEM
   // allocation never waits on another CTA
   static constexpr int SMEM_ALLOC = (SMEM_USED + 1024 > 120 * 1024) ? SMEM_USED + 1024 : 120 * 1024;
-  static constexpr int THREADS = 192;
+  static constexpr int THREADS = 320;
+  static constexpr int W_PROD = 8, W_MMA = 9;
   // TMEM columns
   static constexpr uint32_t T_S0 = 0, T_S1 = 128, T_O = 256, T_P0 = 384, T_P1 = 448;
   static constexpr uint32_t T_COLS = 512;
@@ -72,7 +78,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
   uint32_t* tslot = reinterpret_cast<uint32_t*>(smem + C::MISC_OFF);
   const uint32_t abort_flag = smem_u32(smem + C::MISC_OFF + 4);
-  float* red = reinterpret_cast<float*>(smem + C::MISC_OFF + 16);  // 4 partial sums
+  const uint32_t red = sbase + C::MISC_OFF + 16;  // 8 partial sums of 1/2 l^2
 
   const uint32_t b_q = smem_u32(&bars[0]);
   auto b_kfull = [&](int s) { return smem_u32(&bars[1 + s]); };
@@ -83,6 +89,9 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
   auto b_pfull = [&](int b) { return smem_u32(&bars[3 + 4 * C::NS + b]); };
   auto b_pvdone = [&](int b) { return smem_u32(&bars[5 + 4 * C::NS + b]); };
   const uint32_t b_drain = smem_u32(&bars[7 + 4 * C::NS]);
+  auto b_xch = [&](int b) { return smem_u32(&bars[8 + 4 * C::NS + b]); };
+  const uint32_t b_ep1 = smem_u32(&bars[10 + 4 * C::NS]);
+  const uint32_t b_ep2 = smem_u32(&bars[11 + 4 * C::NS]);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   // head-major order: the query tiles of one (b, h) run side by side and share its K~, V in
@@ -103,14 +112,17 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(b_sfull(b), 1);
-      mbar_init(b_pfull(b), 128);
+      mbar_init(b_pfull(b), 256);
       mbar_init(b_pvdone(b), 1);
+      mbar_init(b_xch(b), 256);
     }
     mbar_init(b_drain, 1);
+    mbar_init(b_ep1, 256);
+    mbar_init(b_ep2, 256);
     abort_set(abort_flag, 0);
     fence_barrier_init();
   }
-  if (warp == 5) {
+  if (warp == C::W_MMA) {
     tmem_alloc(smem_u32(tslot), C::T_COLS);
     tmem_relinquish();
   }
@@ -119,7 +131,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
   tc_fence_after();
   const uint32_t tmem = *tslot;
 
-  if (warp == 4) {
+  if (warp == C::W_PROD) {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
       tma_prefetch(&tm_q);
@@ -155,7 +167,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
           mbar_drain(b_vfull(j % C::NS), (j / C::NS) & 1, lim);
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == C::W_MMA) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, false, false);
@@ -200,61 +212,75 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
       }
     }
   } else {
-    // ------------------------------------------------------------------ softmax warps 0-3
-    const int row = qt * C::BM + tid;
-    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    // ------------------------------------------------------------------ softmax warps 0-7
+    // warp w reaches TMEM lanes 32 (w % 4) ...; warpgroup `half` takes key columns
+    // 64 half .. 64 half + 63 of each tile and head-dimension columns D/2 half .. of O
+    const int r = tid & 127, half = warp >> 2;
+    const int row = qt * C::BM + r;
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t xch = sbase + C::XCH_OFF;
+    constexpr int OH = D / 2;  // O columns per warpgroup
     float m = -INFINITY, l = 0.f;
     bool ok = true;
     for (int j = 0; j < T; ++j) {
       const int sb = j & 1;
       if (!(ok = mbar_wait_warp(b_sfull(sb), (j >> 1) & 1, abort_flag, lim))) break;
       tc_fence_after();
-      float x[128];
+      float x[64];
       {
-        const uint32_t s_addr = tmem + lane_base + (sb ? C::T_S1 : C::T_S0);
-        uint32_t r[4][32];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_ld32(s_addr + 32 * c, r[c]);
+        const uint32_t s_addr = tmem + lane_base + (sb ? C::T_S1 : C::T_S0) + 64 * half;
+        uint32_t r0[32], r1[32];
+        tmem_ld32(s_addr, r0);
+        tmem_ld32(s_addr + 32, r1);
         tmem_wait_ld();
 #pragma unroll
-        for (int c = 0; c < 4; ++c)
-#pragma unroll
-          for (int i = 0; i < 32; ++i) x[32 * c + i] = __uint_as_float(r[c][i]) * p.scale_log2;
+        for (int i = 0; i < 32; ++i) {
+          x[i] = __uint_as_float(r0[i]) * p.scale_log2;
+          x[32 + i] = __uint_as_float(r1[i]) * p.scale_log2;
+        }
       }
-      const int key0 = j * C::BN;
-      if (key0 + C::BN > n || (p.causal && j == qt)) {
+      const int key0 = j * C::BN + 64 * half;
+      if (j * C::BN + C::BN > n || (p.causal && j == qt)) {
 #pragma unroll
-        for (int i = 0; i < 128; ++i) {
+        for (int i = 0; i < 64; ++i) {
           const int key = key0 + i;
           if (key >= n || (p.causal && key > row)) x[i] = -INFINITY;
         }
       }
       float mt = x[0];
 #pragma unroll
-      for (int i = 1; i < 128; ++i) mt = fmaxf(mt, x[i]);
-      const float mnew = fmaxf(m, mt);
+      for (int i = 1; i < 64; ++i) mt = fmaxf(mt, x[i]);
+      // the other half of the row's maximum
+      st_shared_f32(xch + ((sb * 2 + half) * 128 + r) * 4, mt);
+      mbar_arrive(b_xch(sb));
+      if (!(ok = mbar_wait_warp(b_xch(sb), (j >> 1) & 1, abort_flag, lim))) break;
+      const float mo = ld_shared_f32(xch + ((sb * 2 + (half ^ 1)) * 128 + r) * 4);
+      const float mnew = fmaxf(m, fmaxf(mt, mo));
       if (j == 0) {
         m = mnew;
       } else {
+        // both halves of a row take the same decision (same m, same mnew), and warps w and
+        // w + 4 hold the same rows, so the vote agrees across the two warpgroups
         const bool need = mnew > m + 8.f;
         if (__any_sync(0xffffffffu, need)) {
           // O holds P_0..P_{j-1} V: wait for the last product, then rescale in TMEM
           if (!(ok = mbar_wait_warp(b_pvdone((j - 1) & 1), ((j - 1) >> 1) & 1, abort_flag, lim)))
             break;
           tc_fence_after();
-          const float alpha = need ? exp2f(m - mnew) : 1.f;
+          const float alpha = need ? ex2(m - mnew) : 1.f;
           if (need) {
             l *= alpha;
             m = mnew;
           }
 #pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t r[32];
-            tmem_ld32(tmem + lane_base + C::T_O + 32 * c, r);
+          for (int c = 0; c < OH / 32; ++c) {
+            uint32_t rr[32];
+            const uint32_t oa = tmem + lane_base + C::T_O + OH * half + 32 * c;
+            tmem_ld32(oa, rr);
             tmem_wait_ld();
 #pragma unroll
-            for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-            tmem_st32(tmem + lane_base + C::T_O + 32 * c, r);
+            for (int i = 0; i < 32; ++i) rr[i] = __float_as_uint(__uint_as_float(rr[i]) * alpha);
+            tmem_st32(oa, rr);
           }
           tmem_wait_st();
         }
@@ -263,42 +289,43 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
         if (!(ok = mbar_wait_warp(b_pvdone(sb), ((j - 2) >> 1) & 1, abort_flag, lim))) break;
         tc_fence_after();
       }
-      const uint32_t p_addr = tmem + lane_base + (sb ? C::T_P1 : C::T_P0);
       float psum = 0.f;
+      uint32_t pk[32];
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        uint32_t pk[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float p0 = ex2(x[64 * h + 2 * i] - m), p1 = ex2(x[64 * h + 2 * i + 1] - m);
-          psum += p0 + p1;
-          pk[i] = pack_bf16x2(p0, p1);
-        }
-        tmem_st32(p_addr + 32 * h, pk);
+      for (int i = 0; i < 32; ++i) {
+        const float p0 = ex2(x[2 * i] - m), p1 = ex2(x[2 * i + 1] - m);
+        psum += p0 + p1;
+        pk[i] = pack_bf16x2(p0, p1);
       }
+      tmem_st32(tmem + lane_base + (sb ? C::T_P1 : C::T_P0) + 32 * half, pk);
       l += psum;
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(b_pfull(sb));
     }
-    // ---- epilogue
-    float sq = 0.f;
+    // ---- epilogue: each warpgroup finishes its D/2 columns of O
+    float sq = 0.f, dl = 0.f;
     if (ok) ok = mbar_wait_warp(b_pvdone((T - 1) & 1), ((T - 1) >> 1) & 1, abort_flag, lim);
-    if (ok) {
+    st_shared_f32(sbase + C::EPL_OFF + (half * 128 + r) * 4, l);
+    mbar_arrive(b_ep1);
+    const bool ok1 = mbar_wait_warp(b_ep1, 0, abort_flag, lim);
+    const bool vrow = row < n;
+    float l_row = 1.f;
+    if (ok && ok1) {
       tc_fence_after();
-      const float inv_l = 1.f / l;
-      const bool vrow = row < n;
-      const size_t ro = ((size_t)bh * n + row) * D;
-      float dl = 0.f;
+      l_row = ld_shared_f32(sbase + C::EPL_OFF + r * 4) +
+              ld_shared_f32(sbase + C::EPL_OFF + (128 + r) * 4);
+      const float inv_l = 1.f / l_row;
+      const size_t ro = ((size_t)bh * n + row) * D + OH * half;
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t r[32];
-        tmem_ld32(tmem + lane_base + C::T_O + 32 * c, r);
+      for (int c = 0; c < OH / 32; ++c) {
+        uint32_t rr[32];
+        tmem_ld32(tmem + lane_base + C::T_O + OH * half + 32 * c, rr);
         tmem_wait_ld();
         if (vrow) {
           float o[32];
 #pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = __uint_as_float(r[i]) * inv_l;
+          for (int i = 0; i < 32; ++i) o[i] = __uint_as_float(rr[i]) * inv_l;
           uint4* Og = reinterpret_cast<uint4*>(p.O + ro + 32 * c);
 #pragma unroll
           for (int v = 0; v < 4; ++v)
@@ -326,24 +353,29 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
           }
         }
       }
-      if (vrow) {
-        p.lse[(size_t)bh * n + row] = (m + log2f(l)) * kLn2;
-        if (p.E) p.delta[(size_t)bh * n + row] = dl;
-      }
     }
-    if (p.E) {
+    // combine <l, O> of the two halves and the per-warp sums of l^2
+    if (half == 1) st_shared_f32(sbase + C::EPD_OFF + r * 4, dl);
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
-      if (lane == 0) red[warp] = sq;
-      named_bar_sync(1, 128);
-      if (tid == 0)
-        p.loss_part[(size_t)blockIdx.y * gridDim.x + blockIdx.x] =
-            0.5 * ((double)red[0] + (double)red[1] + (double)red[2] + (double)red[3]);
+    for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
+    if (lane == 0) st_shared_f32(red + warp * 4, sq);
+    mbar_arrive(b_ep2);
+    const bool ok2 = mbar_wait_warp(b_ep2, 0, abort_flag, lim);
+    if (ok && ok1 && ok2) {
+      if (half == 0 && vrow) {
+        p.lse[(size_t)bh * n + row] = (m + log2f(l_row)) * kLn2;
+        if (p.E) p.delta[(size_t)bh * n + row] = dl + ld_shared_f32(sbase + C::EPD_OFF + r * 4);
+      }
+      if (p.E && tid == 0) {
+        double t = 0.0;
+        for (int w = 0; w < 8; ++w) t += (double)ld_shared_f32(red + w * 4);
+        p.loss_part[(size_t)blockIdx.y * gridDim.x + blockIdx.x] = 0.5 * t;
+      }
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == C::W_MMA) {
     tc_fence_after();
     tmem_dealloc(tmem, C::T_COLS);
   }
