@@ -7,6 +7,8 @@
 //   P^T    = exp(S^T / sqrt(d) - lse_i)  recomputed softmax s(x) from the stored log-sum-exp
 //   gamma^T = P^T o (beta^T - delta_i)   gamma = diag(s) beta - s s^T beta, with the row sums
 //                                        s_i^T beta_i = <l_i, O_i> = delta_i
+//   (P^T and gamma^T are written to TMEM, where they are the A operands of the next two
+//    products; gamma^T also goes to shared memory as the B operand of dQ~^T)
 //   dV    += P^T l_i                   (accumulated in TMEM over all query tiles)
 //   dK~   += gamma^T Q~_i              (scaled by 1/sqrt(d) and un-rotated at the end)
 //   dQ~_i^T = K~^T gamma^T             (d on TMEM lanes; staged in shared memory and added to
@@ -31,27 +33,26 @@ template <int D>
 struct BwdCfg {
   static constexpr int BK = 128;              // keys per CTA
   static constexpr int BQ = 64;               // query rows per step
-  static constexpr int NSQ = 2;               // query-tile pipeline stages
+  static constexpr int NSQ = 3;               // query-tile pipeline stages
   static constexpr int KB = D / 64;           // 128-byte swizzle blocks per row
   static constexpr int KTILE = BK * D * 2;    // K~ or V tile bytes
   static constexpr int QTILE = BQ * D * 2;    // Q~_i or l_i tile bytes
   static constexpr int KBLK = BK * 128;       // one swizzle block of a 128-row tile
   static constexpr int QBLK = BQ * 128;       // one swizzle block of a 64-row tile
-  static constexpr int PG = BK * BQ * 2;      // P^T or gamma^T buffer bytes (one block)
+  static constexpr int PG = BK * BQ * 2;      // gamma^T buffer bytes (one swizzle block)
   static constexpr int K_OFF = 0;
   static constexpr int V_OFF = K_OFF + KTILE;
   static constexpr int Q_OFF = V_OFF + KTILE;            // NSQ stages
   static constexpr int L_OFF = Q_OFF + NSQ * QTILE;      // NSQ stages
-  static constexpr int P_OFF = L_OFF + NSQ * QTILE;      // 2 buffers
-  static constexpr int G_OFF = P_OFF + 2 * PG;           // 2 buffers
-  static constexpr int DQS_OFF = G_OFF + 2 * PG;          // fp32 [BQ][D] dQ~ staging tile
+  static constexpr int G_OFF = L_OFF + NSQ * QTILE;      // gamma^T, B operand of dQ~^T
+  static constexpr int DQS_OFF = G_OFF + PG;              // fp32 [BQ][D] dQ~ staging tile
   static constexpr int DQS = BQ * D * 4;
   // float [NSQ][BQ][2]: (lse * log2(e), delta) per query row
   static constexpr int LD_OFF = DQS_OFF + DQS;
   static constexpr int BAR_OFF = LD_OFF + NSQ * BQ * 8;
-  // kv_full, q_full[NSQ], q_empty[NSQ], s_full, s_free, pg_full[2], pg_free[2],
-  // dq_full[2], dq_free[2], acc_done, drain, dqs_full, dqs_free
-  static constexpr int NBAR = 1 + 2 * NSQ + 2 + 8 + 2 + 2;
+  // kv_full, q_full[NSQ], q_empty[NSQ], s_full, s_free, pg_full, pg_free, dq_full, dq_free,
+  // acc_done, drain, dqs_full, dqs_free
+  static constexpr int NBAR = 1 + 2 * NSQ + 10;
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
   static constexpr int SMEM_USED = MISC_OFF + 64;
   static constexpr int SMEM_ALLOC =
@@ -59,7 +60,7 @@ struct BwdCfg {
   static constexpr int THREADS = 448;
   static constexpr int W_DRAIN = 8, W_PROD = 12, W_MMA = 13;
   // TMEM columns
-  static constexpr uint32_t T_S = 0, T_B = 64, T_DQ0 = 128, T_DQ1 = 192, T_DK = 256,
+  static constexpr uint32_t T_S = 0, T_B = 64, T_DQ = 128, T_PT = 192, T_GT = 224, T_DK = 256,
                             T_DV = 256 + D;
   static constexpr uint32_t T_COLS = 512;
   static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
@@ -96,14 +97,14 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
   auto b_qempty = [&](int s) { return smem_u32(&bars[1 + C::NSQ + s]); };
   const uint32_t b_sfull = smem_u32(&bars[1 + 2 * C::NSQ]);
   const uint32_t b_sfree = smem_u32(&bars[2 + 2 * C::NSQ]);
-  auto b_pgfull = [&](int b) { return smem_u32(&bars[3 + 2 * C::NSQ + b]); };
-  auto b_pgfree = [&](int b) { return smem_u32(&bars[5 + 2 * C::NSQ + b]); };
-  auto b_dqfull = [&](int b) { return smem_u32(&bars[7 + 2 * C::NSQ + b]); };
-  auto b_dqfree = [&](int b) { return smem_u32(&bars[9 + 2 * C::NSQ + b]); };
-  const uint32_t b_acc = smem_u32(&bars[11 + 2 * C::NSQ]);
-  const uint32_t b_drain = smem_u32(&bars[12 + 2 * C::NSQ]);
-  const uint32_t b_dqsfull = smem_u32(&bars[13 + 2 * C::NSQ]);
-  const uint32_t b_dqsfree = smem_u32(&bars[14 + 2 * C::NSQ]);
+  const uint32_t b_pgfull = smem_u32(&bars[3 + 2 * C::NSQ]);
+  const uint32_t b_pgfree = smem_u32(&bars[4 + 2 * C::NSQ]);
+  const uint32_t b_dqfull = smem_u32(&bars[5 + 2 * C::NSQ]);
+  const uint32_t b_dqfree = smem_u32(&bars[6 + 2 * C::NSQ]);
+  const uint32_t b_acc = smem_u32(&bars[7 + 2 * C::NSQ]);
+  const uint32_t b_drain = smem_u32(&bars[8 + 2 * C::NSQ]);
+  const uint32_t b_dqsfull = smem_u32(&bars[9 + 2 * C::NSQ]);
+  const uint32_t b_dqsfree = smem_u32(&bars[10 + 2 * C::NSQ]);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   // head-major order: the key tiles of one (b, h) run side by side and share its Q~, l and
@@ -124,12 +125,10 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     }
     mbar_init(b_sfull, 1);
     mbar_init(b_sfree, 256);
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(b_pgfull(b), 256);
-      mbar_init(b_pgfree(b), 1);
-      mbar_init(b_dqfull(b), 1);
-      mbar_init(b_dqfree(b), 128);
-    }
+    mbar_init(b_pgfull, 256);
+    mbar_init(b_pgfree, 1);
+    mbar_init(b_dqfull, 1);
+    mbar_init(b_dqfree, 128);
     mbar_init(b_acc, 1);
     mbar_init(b_drain, 1);
     mbar_init(b_dqsfull, 128);
@@ -224,31 +223,33 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
           if (!(ok = mbar_wait(b_sfree, ii & 1, abort_flag, lim))) break;
           if (!(ok = issue_sb(ii + 1))) break;
         }
-        const int pb = ii & 1, s = ii % C::NSQ;
-        if (!(ok = mbar_wait(b_pgfull(pb), (ii >> 1) & 1, abort_flag, lim))) break;
+        const int s = ii % C::NSQ;
+        if (!(ok = mbar_wait(b_pgfull, ii & 1, abort_flag, lim))) break;
         tc_fence_after();
-        const uint32_t pt = sbase + C::P_OFF + pb * C::PG;
-        const uint32_t gt = sbase + C::G_OFF + pb * C::PG;
+        const uint32_t gt = sbase + C::G_OFF;
         const uint32_t qb = sbase + C::Q_OFF + s * C::QTILE;
         const uint32_t lb = sbase + C::L_OFF + s * C::QTILE;
-        // dV += P^T l_i, dK += gamma^T Q~_i   (M = 128 keys, N = D, K = 64 queries)
+        // dV += P^T l_i, dK += gamma^T Q~_i: M = 128 keys, N = D, K = 64 queries, with
+        // P^T and gamma^T read from TMEM (two bf16 per column, 8 columns per K step)
 #pragma unroll
         for (int kk = 0; kk < C::BQ / 16; ++kk) {
-          mma_ss(tmem + C::T_DV, sw128_desc(pt + kk * 32, 16, 1024),
+          mma_ts(tmem + C::T_DV, tmem + C::T_PT + kk * 8,
                  sw128_desc(lb + kk * 2048, C::QBLK, 1024), idesc_kv, (ii > 0 || kk > 0));
-          mma_ss(tmem + C::T_DK, sw128_desc(gt + kk * 32, 16, 1024),
+          mma_ts(tmem + C::T_DK, tmem + C::T_GT + kk * 8,
                  sw128_desc(qb + kk * 2048, C::QBLK, 1024), idesc_kv, (ii > 0 || kk > 0));
         }
-        // dQ~_i^T = K~^T gamma^T   (M = D, N = 64 queries, K = 128 keys)
-        if (!(ok = mbar_wait(b_dqfree(pb), ((ii >> 1) & 1) ^ 1, abort_flag, lim))) break;
-        tc_fence_after();
-        const uint32_t dq = tmem + (pb ? C::T_DQ1 : C::T_DQ0);
+        // dQ~_i^T = K~^T gamma^T   (M = D, N = 64 queries, K = 128 keys), once the drain has
+        // read the previous tile's dQ~ out of TMEM
+        if (ii > 0) {
+          if (!(ok = mbar_wait(b_dqfree, (ii - 1) & 1, abort_flag, lim))) break;
+          tc_fence_after();
+        }
 #pragma unroll
         for (int kk = 0; kk < C::BK / 16; ++kk)
-          mma_ss(dq, sw128_desc(ka + kk * 2048, C::KBLK, 1024),
+          mma_ss(tmem + C::T_DQ, sw128_desc(ka + kk * 2048, C::KBLK, 1024),
                  sw128_desc(gt + kk * 2048, C::KBLK, 1024), idesc_dq, kk > 0);
-        mma_commit(b_dqfull(pb));
-        mma_commit(b_pgfree(pb));
+        mma_commit(b_dqfull);
+        mma_commit(b_pgfree);
         mma_commit(b_qempty(s));
       }
       if (ok) {
@@ -279,36 +280,40 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       tmem_wait_ld();
       tc_fence_before();
       mbar_arrive(b_sfree);
-      const int pb = ii & 1;
-      if (!(ok = mbar_wait_warp(b_pgfree(pb), ((ii >> 1) & 1) ^ 1, abort_flag, lim))) break;
-      const uint32_t prow = sbase + C::P_OFF + pb * C::PG;
-      const uint32_t grow = sbase + C::G_OFF + pb * C::PG;
       const uint32_t ld_row = sbase + C::LD_OFF + (stg * C::BQ + 32 * half) * 8;
       const int qh = q0 + 32 * half;
       const bool full = key < n && qh + 32 <= n && (!p.causal || key <= qh);
+      uint32_t pw[16], gw[16];
 #pragma unroll
-      for (int c8 = 0; c8 < 4; ++c8) {
-        uint32_t pw[4], gw[4];
-#pragma unroll
-        for (int h = 0; h < 4; ++h) {
-          const int c = c8 * 8 + h * 2;
-          // (lse_c, delta_c, lse_c+1, delta_c+1)
-          const float4 lz = ld_shared_v4f(ld_row + (c >> 1) * 16);
-          const int q = qh + c;
-          const bool v0 = full || (key < n && q < n && (!p.causal || key <= q));
-          const bool v1 = full || (key < n && q + 1 < n && (!p.causal || key <= q + 1));
-          const float p0 = v0 ? ex2(__uint_as_float(sr[c]) * p.scale_log2 - lz.x) : 0.f;
-          const float p1 = v1 ? ex2(__uint_as_float(sr[c + 1]) * p.scale_log2 - lz.z) : 0.f;
-          pw[h] = pack_bf16x2(p0, p1);
-          gw[h] = pack_bf16x2(p0 * (__uint_as_float(br[c]) - lz.y),
-                              p1 * (__uint_as_float(br[c + 1]) - lz.w));
-        }
-        const uint32_t off = sw128_offset(row, 4 * half + c8);
-        st_shared_v4(prow + off, pw[0], pw[1], pw[2], pw[3]);
-        st_shared_v4(grow + off, gw[0], gw[1], gw[2], gw[3]);
+      for (int h = 0; h < 16; ++h) {
+        const int c = 2 * h;
+        // (lse_c, delta_c, lse_c+1, delta_c+1)
+        const float4 lz = ld_shared_v4f(ld_row + h * 16);
+        const int q = qh + c;
+        const bool v0 = full || (key < n && q < n && (!p.causal || key <= q));
+        const bool v1 = full || (key < n && q + 1 < n && (!p.causal || key <= q + 1));
+        const float p0 = v0 ? ex2(__uint_as_float(sr[c]) * p.scale_log2 - lz.x) : 0.f;
+        const float p1 = v1 ? ex2(__uint_as_float(sr[c + 1]) * p.scale_log2 - lz.z) : 0.f;
+        pw[h] = pack_bf16x2(p0, p1);
+        gw[h] = pack_bf16x2(p0 * (__uint_as_float(br[c]) - lz.y),
+                            p1 * (__uint_as_float(br[c + 1]) - lz.w));
       }
+      // the previous tile's products have read P^T, gamma^T (TMEM) and gamma^T (smem)
+      if (ii > 0) {
+        if (!(ok = mbar_wait_warp(b_pgfree, (ii - 1) & 1, abort_flag, lim))) break;
+        tc_fence_after();
+      }
+      tmem_st16(tmem + lane_base + C::T_PT + 16 * half, pw);
+      tmem_st16(tmem + lane_base + C::T_GT + 16 * half, gw);
+      const uint32_t gsm = sbase + C::G_OFF;
+#pragma unroll
+      for (int c8 = 0; c8 < 4; ++c8)
+        st_shared_v4(gsm + sw128_offset(row, 4 * half + c8), gw[4 * c8], gw[4 * c8 + 1],
+                     gw[4 * c8 + 2], gw[4 * c8 + 3]);
+      tmem_wait_st();
       fence_proxy_async_smem();
-      mbar_arrive(b_pgfull(pb));
+      tc_fence_before();
+      mbar_arrive(b_pgfull);
     }
     // ---- dK = rot^-1(scale * sum gamma^T Q~) (warps 0-3), dV = sum P^T l (warps 4-7):
     //      one key row per thread
@@ -354,16 +359,15 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     const uint32_t stage = sbase + C::DQS_OFF;
     const bool issuer = tid == 32 * C::W_DRAIN;
     for (int ii = 0; ii < NI; ++ii) {
-      const int pb = ii & 1;
-      if (!mbar_wait_warp(b_dqfull(pb), (ii >> 1) & 1, abort_flag, lim)) break;
+      if (!mbar_wait_warp(b_dqfull, ii & 1, abort_flag, lim)) break;
       tc_fence_after();
       uint32_t r0[32], r1[32];
-      const uint32_t dq = tmem + lane_base + (pb ? C::T_DQ1 : C::T_DQ0);
+      const uint32_t dq = tmem + lane_base + C::T_DQ;
       tmem_ld32(dq, r0);
       tmem_ld32(dq + 32, r1);
       tmem_wait_ld();
       tc_fence_before();
-      mbar_arrive(b_dqfree(pb));
+      mbar_arrive(b_dqfree);
       // the staging tile is free once the previous bulk reduction has read it
       if (!mbar_wait_warp(b_dqsfree, (ii & 1) ^ 1, abort_flag, lim)) break;
       if (has_row) {
