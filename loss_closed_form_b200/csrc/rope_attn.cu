@@ -346,11 +346,19 @@ ra_status tc_project(const ra_problem* p, const Layout& L, void* ws, cudaStream_
   pp.out[1] = at<__nv_bfloat16>(ws, L.kt);
   pp.out[2] = at<__nv_bfloat16>(ws, L.v);
   pp.n = n;
+  pp.B = p->B;
   pp.H = p->H;
+  pp.nrt = (n + C::BM - 1) / C::BM;
+  // persistent CTAs over the 128-row tiles of one (z, h): about two waves of 148 CTAs
+  const long tiles = (long)p->B * pp.nrt;
+  long chunks = (2 * 148 + 3 * p->H - 1) / (3 * p->H);
+  chunks = chunks < 1 ? 1 : (chunks > tiles ? tiles : chunks);
+  pp.tiles_per_cta = (int)((tiles + chunks - 1) / chunks);
+  chunks = (tiles + pp.tiles_per_cta - 1) / pp.tiles_per_cta;
   pp.limit_ns = wait_limit_ns();
   auto k = proj_rope_tc_kernel<D>;
   cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_ALLOC);
-  dim3 grid(BH, (n + C::BM - 1) / C::BM, 3);
+  dim3 grid((unsigned)chunks, p->H, 3);
   Launch l(K_PROJ_TC, st);
   k<<<grid, C::THREADS, C::SMEM_ALLOC, st>>>(a1, a2, a3, w1, w2, w3, pp);
   return launch_status();

@@ -235,10 +235,12 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
         tmem_wait_ld();
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
-          x[i] = __uint_as_float(r0[i]) * p.scale_log2;
-          x[32 + i] = __uint_as_float(r1[i]) * p.scale_log2;
+          x[i] = __uint_as_float(r0[i]);
+          x[32 + i] = __uint_as_float(r1[i]);
         }
       }
+      // raw scores: the scale log2(e)/sqrt(d) > 0 is applied to the row maximum and folded
+      // into the exponent's argument
       const int key0 = j * C::BN + 64 * half;
       if (j * C::BN + C::BN > n || (p.causal && j == qt)) {
 #pragma unroll
@@ -255,7 +257,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
       mbar_arrive(b_xch(sb));
       if (!(ok = mbar_wait_warp(b_xch(sb), (j >> 1) & 1, abort_flag, lim))) break;
       const float mo = ld_shared_f32(xch + ((sb * 2 + (half ^ 1)) * 128 + r) * 4);
-      const float mnew = fmaxf(m, fmaxf(mt, mo));
+      const float mnew = fmaxf(m, fmaxf(mt, mo) * p.scale_log2);
       if (j == 0) {
         m = mnew;
       } else {
@@ -293,7 +295,8 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
       uint32_t pk[32];
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
-        const float p0 = ex2(x[2 * i] - m), p1 = ex2(x[2 * i + 1] - m);
+        const float p0 = ex2(fmaf(x[2 * i], p.scale_log2, -m));
+        const float p1 = ex2(fmaf(x[2 * i + 1], p.scale_log2, -m));
         psum += p0 + p1;
         pk[i] = pack_bf16x2(p0, p1);
       }

@@ -22,29 +22,35 @@ template <int D>
 struct ProjCfg {
   static constexpr int BM = 128;
   static constexpr int KB = D / 64;
+  static constexpr int NS = 4;               // A-tile stages
   static constexpr int ATILE = BM * D * 2;
   static constexpr int WTILE = D * D * 2;
-  static constexpr int ABLK = BM * 128;  // [128 rows][64 cols] block
-  static constexpr int WBLK = D * 128;   // [D rows][64 cols] block
-  static constexpr int A_OFF = 0;
-  static constexpr int W_OFF = ATILE;
-  static constexpr int BAR_OFF = W_OFF + WTILE;  // full, mma_done
-  static constexpr int MISC_OFF = BAR_OFF + 16;
+  static constexpr int ABLK = BM * 128;      // [128 rows][64 cols] block
+  static constexpr int WBLK = D * 128;       // [D rows][64 cols] block
+  static constexpr int W_OFF = 0;
+  static constexpr int A_OFF = WTILE;
+  static constexpr int BAR_OFF = A_OFF + NS * ATILE;
+  // w_full, a_full[NS], a_empty[NS], acc_full[2], acc_empty[2], drain
+  static constexpr int NBAR = 1 + 2 * NS + 4 + 1;
+  static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
   static constexpr int SMEM_ALLOC = MISC_OFF + 16 + 1024;
-  static constexpr int THREADS = 128;
-  static constexpr uint32_t T_COLS = D;
+  static constexpr int THREADS = 192;        // warps 0-3 epilogue, 4 TMA, 5 MMA
+  static constexpr uint32_t T_COLS = 2 * D;  // double-buffered accumulator
 };
 
 struct ProjParams {
-  const float2* tab;         // [n][d/2] (cos, sin)
-  __nv_bfloat16* out[3];     // Q~, K~, V: [BH][n][d]
-  int n, H;
+  const float2* tab;       // [n][d/2] (cos, sin)
+  __nv_bfloat16* out[3];   // Q~, K~, V: [BH][n][d]
+  int n, B, H, nrt;        // nrt = 128-row tiles per instance
+  int tiles_per_cta;
   unsigned long long limit_ns;
 };
 
-// grid (BH, ceil(n/128), 3): z = 0 (Q, rotated), 1 (K, rotated), 2 (V)
+// grid (chunks, H, 3): the CTA (c, h, z) projects tiles t = b * nrt + rt in
+// [c * tiles_per_cta, ...) of head h with W_z[h] loaded once; z = 0 (Q, rotated),
+// 1 (K, rotated), 2 (V).
 template <int D>
-__global__ void __launch_bounds__(ProjCfg<D>::THREADS)
+__global__ void __launch_bounds__(ProjCfg<D>::THREADS, 1)
 proj_rope_tc_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_constant__ CUtensorMap tm_a2,
                     const __grid_constant__ CUtensorMap tm_a3, const __grid_constant__ CUtensorMap tm_w1,
                     const __grid_constant__ CUtensorMap tm_w2, const __grid_constant__ CUtensorMap tm_w3,
@@ -57,19 +63,34 @@ proj_rope_tc_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_cons
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
   uint32_t* tslot = reinterpret_cast<uint32_t*>(smem + C::MISC_OFF);
   const uint32_t abort_flag = smem_u32(smem + C::MISC_OFF + 4);
-  const uint32_t b_full = smem_u32(&bars[0]), b_mma = smem_u32(&bars[1]);
-  const int tid = threadIdx.x, warp = tid >> 5;
-  const int bh = blockIdx.x, rt = blockIdx.y, z = blockIdx.z, h = bh % p.H;
+  const uint32_t b_w = smem_u32(&bars[0]);
+  auto b_afull = [&](int s) { return smem_u32(&bars[1 + s]); };
+  auto b_aempty = [&](int s) { return smem_u32(&bars[1 + C::NS + s]); };
+  auto b_accfull = [&](int b) { return smem_u32(&bars[1 + 2 * C::NS + b]); };
+  auto b_accempty = [&](int b) { return smem_u32(&bars[3 + 2 * C::NS + b]); };
+  const uint32_t b_drain = smem_u32(&bars[5 + 2 * C::NS]);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int h = blockIdx.y, z = blockIdx.z;
   const CUtensorMap* tma = z == 0 ? &tm_a1 : z == 1 ? &tm_a2 : &tm_a3;
   const CUtensorMap* tmw = z == 0 ? &tm_w1 : z == 1 ? &tm_w2 : &tm_w3;
+  const int t0 = blockIdx.x * p.tiles_per_cta;
+  const int NT = min(p.tiles_per_cta, p.B * p.nrt - t0);
   const uint64_t lim = p.limit_ns;
   if (tid == 0) {
-    mbar_init(b_full, 1);
-    mbar_init(b_mma, 1);
+    mbar_init(b_w, 1);
+    for (int s = 0; s < C::NS; ++s) {
+      mbar_init(b_afull(s), 1);
+      mbar_init(b_aempty(s), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(b_accfull(b), 1);
+      mbar_init(b_accempty(b), 128);
+    }
+    mbar_init(b_drain, 1);
     abort_set(abort_flag, 0);
     fence_barrier_init();
   }
-  if (warp == 0) {
+  if (warp == 5) {
     tmem_alloc(smem_u32(tslot), C::T_COLS);
     tmem_relinquish();
   }
@@ -77,62 +98,97 @@ proj_rope_tc_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_cons
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tslot;
-  bool ok = true;
-  if (tid == 0) {
-    mbar_expect_tx(b_full, C::ATILE + C::WTILE);
-    for (int b = 0; b < C::KB; ++b) {
-      tma_load_3d(sbase + C::A_OFF + b * C::ABLK, tma, b_full, 64 * b, rt * C::BM, bh);
-      tma_load_3d(sbase + C::W_OFF + b * C::WBLK, tmw, b_full, 64 * b, 0, h);
+  if (warp == 4) {
+    // ------------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      mbar_expect_tx(b_w, C::WTILE);
+      for (int b = 0; b < C::KB; ++b)
+        tma_load_3d(sbase + C::W_OFF + b * C::WBLK, tmw, b_w, 64 * b, 0, h);
+      int last = -1;
+      for (int t = 0; t < NT; ++t) {
+        const int s = t % C::NS;
+        if (!mbar_wait(b_aempty(s), ((t / C::NS) & 1) ^ 1, abort_flag, lim)) break;
+        const int tt = t0 + t, b = tt / p.nrt, rt = tt - b * p.nrt;
+        mbar_expect_tx(b_afull(s), C::ATILE);
+        for (int kb = 0; kb < C::KB; ++kb)
+          tma_load_3d(sbase + C::A_OFF + s * C::ATILE + kb * C::ABLK, tma, b_afull(s), 64 * kb,
+                      rt * C::BM, b * p.H + h);
+        last = t;
+      }
+      if (abort_get(abort_flag)) {
+        mbar_drain(b_w, 0, lim);
+        for (int t = (last - C::NS + 1 > 0 ? last - C::NS + 1 : 0); t <= last; ++t)
+          mbar_drain(b_afull(t % C::NS), (t / C::NS) & 1, lim);
+      }
     }
-    ok = mbar_wait(b_full, 0, abort_flag, lim);
-    tc_fence_after();
-    if (ok) {
+  } else if (warp == 5) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
       constexpr uint32_t idesc = idesc_bf16_f32(128, D, false, true);
+      bool ok = mbar_wait(b_w, 0, abort_flag, lim);
+      for (int t = 0; ok && t < NT; ++t) {
+        const int s = t % C::NS, ab = t & 1;
+        if (!(ok = mbar_wait(b_afull(s), (t / C::NS) & 1, abort_flag, lim))) break;
+        if (!(ok = mbar_wait(b_accempty(ab), ((t >> 1) & 1) ^ 1, abort_flag, lim))) break;
+        tc_fence_after();
+        const uint32_t a = sbase + C::A_OFF + s * C::ATILE;
 #pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk)
-        mma_ss(tmem, sw128_desc(sbase + C::A_OFF + (kk >> 2) * C::ABLK + (kk & 3) * 32, 16, 1024),
-               sw128_desc(sbase + C::W_OFF + kk * 2048, C::WBLK, 1024), idesc, kk > 0);
+        for (int kk = 0; kk < D / 16; ++kk)
+          mma_ss(tmem + ab * D, sw128_desc(a + (kk >> 2) * C::ABLK + (kk & 3) * 32, 16, 1024),
+                 sw128_desc(sbase + C::W_OFF + kk * 2048, C::WBLK, 1024), idesc, kk > 0);
+        mma_commit(b_accfull(ab));
+        mma_commit(b_aempty(s));
+      }
+      if (!ok) {
+        mma_commit(b_drain);
+        mbar_drain(b_drain, 0, lim);
+      }
     }
-    mma_commit(b_mma);  // also the drain on failure: arrives once nothing is in flight
-    if (!ok) mbar_drain(b_full, 0, lim);
-  }
-  __syncwarp();
-  ok = mbar_wait_warp(b_mma, 0, abort_flag, lim) && !abort_get(abort_flag);
-  tc_fence_after();
-  if (ok) {
-    const int row = rt * C::BM + tid;
+  } else {
+    // ------------------------------------------------------------------ epilogue (warps 0-3)
     const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-    const bool vrow = row < p.n;
-    __nv_bfloat16* out = p.out[z] + ((size_t)bh * p.n + row) * D;
-    const float2* tr = p.tab + (size_t)(vrow ? row : 0) * (D / 2);
+    __nv_bfloat16* out_base = p.out[z];
+    for (int t = 0; t < NT; ++t) {
+      const int ab = t & 1;
+      if (!mbar_wait_warp(b_accfull(ab), (t >> 1) & 1, abort_flag, lim)) break;
+      tc_fence_after();
+      const int tt = t0 + t, b = tt / p.nrt, rt = tt - b * p.nrt;
+      const int row = rt * C::BM + tid;
+      const bool vrow = row < p.n;
+      uint32_t r[D];
 #pragma unroll
-    for (int c = 0; c < D / 32; ++c) {
-      uint32_t r[32];
-      tmem_ld32(tmem + lane_base + 32 * c, r);
+      for (int c = 0; c < D / 32; ++c)
+        tmem_ld32(tmem + lane_base + ab * D + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&r[32 * c]));
       tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(b_accempty(ab));
       if (vrow) {
-        uint32_t w[16];
+        __nv_bfloat16* out = out_base + ((size_t)(b * p.H + h) * p.n + row) * D;
+        const float4* tr = reinterpret_cast<const float4*>(p.tab + (size_t)row * (D / 2));
 #pragma unroll
-        for (int k = 0; k < 16; ++k) {
-          float x0 = __uint_as_float(r[2 * k]), x1 = __uint_as_float(r[2 * k + 1]);
-          if (z < 2) {
-            const float2 cs = tr[16 * c + k];
-            const float y0 = x0 * cs.x - x1 * cs.y;
-            const float y1 = x0 * cs.y + x1 * cs.x;
-            x0 = y0;
-            x1 = y1;
+        for (int c = 0; c < D / 8; ++c) {  // 8 columns = 4 pairs = one 16-byte store
+          uint32_t w[4];
+#pragma unroll
+          for (int k2 = 0; k2 < 2; ++k2) {
+            float x0 = __uint_as_float(r[8 * c + 4 * k2]), x1 = __uint_as_float(r[8 * c + 4 * k2 + 1]);
+            float x2 = __uint_as_float(r[8 * c + 4 * k2 + 2]), x3 = __uint_as_float(r[8 * c + 4 * k2 + 3]);
+            if (z < 2) {
+              const float4 cs = tr[2 * c + k2];  // (cos, sin) of two consecutive pairs
+              const float y0 = x0 * cs.x - x1 * cs.y, y1 = x0 * cs.y + x1 * cs.x;
+              const float y2 = x2 * cs.z - x3 * cs.w, y3 = x2 * cs.w + x3 * cs.z;
+              x0 = y0; x1 = y1; x2 = y2; x3 = y3;
+            }
+            w[2 * k2] = pack_bf16x2(x0, x1);
+            w[2 * k2 + 1] = pack_bf16x2(x2, x3);
           }
-          w[k] = pack_bf16x2(x0, x1);
+          reinterpret_cast<uint4*>(out)[c] = make_uint4(w[0], w[1], w[2], w[3]);
         }
-        uint4* o = reinterpret_cast<uint4*>(out + 32 * c);
-#pragma unroll
-        for (int v = 0; v < 4; ++v) o[v] = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
       }
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) {
+  if (warp == 5) {
     tc_fence_after();
     tmem_dealloc(tmem, C::T_COLS);
   }

@@ -158,9 +158,23 @@ __global__ void probe_timeout_kernel(unsigned long long limit_ns, int* waited_ok
   if (threadIdx.x == 0) *waited_ok = ok ? 1 : 0;
 }
 
+__global__ void probe_exp2_kernel(const float* __restrict__ x, float* __restrict__ poly,
+                                  float* __restrict__ ref, int n) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  poly[i] = exp2_poly(x[i]);
+  ref[i] = exp2f(x[i]);
+}
+
 }  // namespace
 
 extern "C" {
+
+// exp2_poly and CUDA's exp2f on the same inputs (device buffers of n floats).
+int probe_exp2(const float* x, float* poly, float* ref, int n) {
+  probe_exp2_kernel<<<(n + 255) / 256, 256>>>(x, poly, ref, n);
+  return (int)cudaGetLastError();
+}
 
 int probe_mma(const void* A, const void* B, float* D, int M, int N, int K, int a_mn, int b_mn,
               int a_tmem, void* stream) {

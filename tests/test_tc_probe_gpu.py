@@ -56,3 +56,22 @@ def test_bounded_wait_gives_up(probe):
     # the context is still usable
     x = torch.ones(4, device="cuda")
     assert float(x.sum()) == 4.0
+
+
+def test_exp2_poly_against_cuda_exp2f(probe):
+    """The FMA-pipe 2^x used for part of the softmax exponentials, against exp2f."""
+    x = torch.cat([torch.linspace(-126.0, 8.0, 1 << 20, device="cuda"),
+                   torch.tensor([0.0, -0.5, 0.5, -1e-7, 7.99], device="cuda")])
+    poly = torch.empty_like(x)
+    ref = torch.empty_like(x)
+    assert probe.probe_exp2(ctypes.c_void_p(x.data_ptr()), ctypes.c_void_p(poly.data_ptr()),
+                            ctypes.c_void_p(ref.data_ptr()), x.numel()) == 0
+    torch.cuda.synchronize()
+    rel = ((poly.double() - ref.double()).abs() / ref.double()).max().item()
+    assert rel <= 4e-6, rel
+    low = torch.tensor([-127.0, -200.0, float("-inf")], device="cuda")
+    out = torch.empty_like(low)
+    probe.probe_exp2(ctypes.c_void_p(low.data_ptr()), ctypes.c_void_p(out.data_ptr()),
+                     ctypes.c_void_p(torch.empty_like(low).data_ptr()), 3)
+    torch.cuda.synchronize()
+    assert torch.isfinite(out).all() and (out >= 0).all() and (out <= 2.0 ** -125).all()

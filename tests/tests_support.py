@@ -11,4 +11,6 @@ def probe_lib():
     lib.probe_mma.restype = ctypes.c_int
     lib.probe_timeout.argtypes = [ctypes.c_ulonglong, ctypes.POINTER(ctypes.c_int)]
     lib.probe_timeout.restype = ctypes.c_int
+    lib.probe_exp2.argtypes = [vp, vp, vp, ctypes.c_int]
+    lib.probe_exp2.restype = ctypes.c_int
     return lib
