@@ -163,8 +163,9 @@ Layout make_layout(const ra_problem* p) {
     L.chunk = (int)((rows + ns - 1) / ns);
   }
   L.nparts_pre = (int)(((n + 31) / 32) * B * H);
-  L.nparts_fwd = p->dtype == RA_BF16 ? (int)(((n + 127) / 128) * B * H) : L.nparts_pre;
-  L.nparts = L.nparts_pre;
+  // the tensor-core forward writes four partial sums per 128-row query tile
+  L.nparts_fwd = p->dtype == RA_BF16 ? (int)(((n + 127) / 128) * B * H * 4) : L.nparts_pre;
+  L.nparts = L.nparts_pre > L.nparts_fwd ? L.nparts_pre : L.nparts_fwd;
   size_t off = 0;
   auto take = [&](size_t bytes) {
     size_t o = off;
@@ -430,12 +431,13 @@ ra_status tc_fwd_launch(const ra_problem* p, const Layout& L, void* O, float* ls
   fp.n = n;
   fp.BH = BH;
   fp.nq = (n + C::BM - 1) / C::BM;
+  fp.npair = (fp.nq + 1) / 2;
   fp.causal = p->causal;
   fp.scale_log2 = ra::kLog2e / sqrtf((float)D);
   fp.limit_ns = wait_limit_ns();
   auto k = attn_fwd_tc_kernel<D>;
   cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_ALLOC);
-  dim3 grid(fp.nq, BH);
+  dim3 grid(fp.npair, BH);
   Launch l(K_FWD_TC, st);
   k<<<grid, C::THREADS, C::SMEM_ALLOC, st>>>(mq, mk, mv, fp);
   return RA_OK;

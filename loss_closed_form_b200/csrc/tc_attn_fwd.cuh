@@ -1,22 +1,29 @@
-// Tensor-core forward: one CTA per 128-row query tile of one (b, h) instance.
+// Tensor-core forward: one CTA per pair of 128-row query tiles of one (b, h) instance.
 //
-//   S_j = Q~ K~_j^T                 (tcgen05, K-major x K-major, fp32 in TMEM, double-buffered)
-//   online softmax over key tiles    (one query row per thread; rows = TMEM lanes)
-//   P_j -> TMEM as bf16, O += P_j V_j (tcgen05 with A read from TMEM, V as an MN-major B)
+//   S_t,j = Q~_t K~_j^T               (tcgen05, K-major x K-major, fp32 in TMEM)
+//   online softmax over key tiles     (one query row per thread; rows = TMEM lanes)
+//   P_t,j -> TMEM as bf16 over S_t,j, O_t += P_t,j V_j (tcgen05, A read from TMEM)
 //   epilogue: O = acc / l, lse, l = O - E, delta_i = <l_i, O_i>, partial 1/2 sum l^2
 //
 // Definitions: s = softmax(Q~ K~^T / sqrt(d)) and O = s V are exact attention D^-1 A V
 // ("HyperAttention" article, section 方法の概要); l = O - E is the error term l(x) of
 // "RoPE Attention kan bijna lineair worden getraind" (Methodologie 1).
 //
+// The two query tiles t = 0, 1 share every K~ / V tile and alternate on the tensor cores:
+// while warpgroup t turns S_t,j into P_t,j, the MMA warp runs the other tile's products, so
+// the exponentials of one tile overlap the matrix products of the other.  TMEM holds S_0,
+// S_1, O_0, O_1 (4 x 128 columns); P_t,j is written over the first 64 columns of S_t,j, and
+// S_t,j+1 is issued only once the product that reads P_t,j has completed.
+//
 // Rescaling of the accumulator is deferred while a row's running maximum grows by at most
 // 2^8 (log2 units): O and l keep one common reference, so the final O / l is unchanged and
-// P stays <= 256 in bf16.
+// P stays <= 256 in bf16.  The row maximum is taken on raw scores; the scale
+// log2(e)/sqrt(d) > 0 is applied to it and folded into each exponent's FFMA.
 //
-// Warp roles (320 threads): warps 0-7 softmax + epilogue (two warpgroups over the same 128
-// query rows, each taking 64 of the 128 key columns of a tile; the row maximum, row sum and
-// <l, O> are combined through shared memory), warp 8 TMA producer, warp 9 MMA issuer and
-// TMEM owner.
+// Warp roles (384 threads): warps 0-3 softmax + epilogue of query tile 0, warps 4-7 of
+// query tile 1, warp 8 TMA producer, warp 9 MMA issuer and TMEM owner, warps 10-11 idle.
+// The third warpgroup hands registers to the two softmax warpgroups (setmaxnreg): a thread
+// there holds a whole 128-column row of scores.
 #pragma once
 #include "tc_ptx.cuh"
 
@@ -27,30 +34,32 @@ template <int D>
 struct FwdCfg {
   static constexpr int BM = 128;               // query rows per tile
   static constexpr int BN = 128;               // keys per tile
-  static constexpr int NS = 2;                 // K / V pipeline stages
+  static constexpr int NS = D == 64 ? 4 : 2;   // K / V pipeline stages
   static constexpr int KB = D / 64;            // 128-byte swizzle blocks per row
   static constexpr int TILE = 128 * D * 2;     // bytes of a 128 x D bf16 tile
   static constexpr int BLK = 128 * 128;        // bytes of one 128-row swizzle block
-  static constexpr int Q_OFF = 0;
-  static constexpr int K_OFF = Q_OFF + TILE;
+  static constexpr int Q_OFF = 0;              // two query tiles
+  static constexpr int K_OFF = Q_OFF + 2 * TILE;
   static constexpr int V_OFF = K_OFF + NS * TILE;
   static constexpr int BAR_OFF = V_OFF + NS * TILE;
   // barriers: q_full, k_full[NS], k_empty[NS], v_full[NS], v_empty[NS], s_full[2],
-  //           p_full[2], pv_done[2], drain, xch[2], ep1, ep2
-  static constexpr int NBAR = 1 + 4 * NS + 6 + 1 + 4;
-  static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;  // tmem slot, abort flag, 8 partial sums
-  static constexpr int XCH_OFF = MISC_OFF + 64;        // float [2 buffers][2 halves][128 rows]
-  static constexpr int EPL_OFF = XCH_OFF + 2 * 2 * 128 * 4;  // float [2 halves][128]: row sums
-  static constexpr int EPD_OFF = EPL_OFF + 2 * 128 * 4;      // float [128]: <l, O> of half 1
-  static constexpr int SMEM_USED = EPD_OFF + 128 * 4;
+  //           p_full[2], pv_done[2], drain
+  static constexpr int NBAR = 1 + 4 * NS + 6 + 1;
+  static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;  // tmem slot, abort flag
+  static constexpr int SMEM_USED = MISC_OFF + 16;
   // at least half of the SM's shared memory: one CTA per SM, so the 512-column TMEM
   // allocation never waits on another CTA
   static constexpr int SMEM_ALLOC = (SMEM_USED + 1024 > 120 * 1024) ? SMEM_USED + 1024 : 120 * 1024;
-  static constexpr int THREADS = 320;
+  static constexpr int THREADS = 384;
   static constexpr int W_PROD = 8, W_MMA = 9;
-  // TMEM columns
-  static constexpr uint32_t T_S0 = 0, T_S1 = 128, T_O = 256, T_P0 = 384, T_P1 = 448;
-  static constexpr uint32_t T_COLS = 512;
+  // registers per thread after the hand-over: 256 x REG_SOFTMAX + 128 x REG_OTHER must not
+  // exceed the 384 x 168 the CTA is launched with
+  static constexpr int REG_SOFTMAX = 216, REG_OTHER = 64;
+  static_assert(256 * REG_SOFTMAX + 128 * REG_OTHER <= 384 * 168, "register hand-over");
+  // TMEM columns: S_t at 128 t (P_t over its first 64 columns), O_t at 256 + 128 t
+  static constexpr uint32_t T_S0 = 0, T_O0 = 256, T_COLS = 512;
+  // loss partial sums written per query tile (one per softmax warp)
+  static constexpr int LOSS_PARTS = 4;
 };
 
 struct FwdParams {
@@ -59,8 +68,8 @@ struct FwdParams {
   float* lse;              // [BH][n]
   __nv_bfloat16* ell;      // [BH][n][d] (with E)
   float* delta;            // [BH][n] (with E)
-  double* loss_part;       // [BH * nq] (with E)
-  int n, BH, nq, causal;
+  double* loss_part;       // [BH][nq][4] (with E)
+  int n, BH, nq, npair, causal;
   float scale_log2;        // log2(e) / sqrt(d)
   unsigned long long limit_ns;
 };
@@ -78,28 +87,28 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
   uint32_t* tslot = reinterpret_cast<uint32_t*>(smem + C::MISC_OFF);
   const uint32_t abort_flag = smem_u32(smem + C::MISC_OFF + 4);
-  const uint32_t red = sbase + C::MISC_OFF + 16;  // 8 partial sums of 1/2 l^2
 
   const uint32_t b_q = smem_u32(&bars[0]);
   auto b_kfull = [&](int s) { return smem_u32(&bars[1 + s]); };
   auto b_kempty = [&](int s) { return smem_u32(&bars[1 + C::NS + s]); };
   auto b_vfull = [&](int s) { return smem_u32(&bars[1 + 2 * C::NS + s]); };
   auto b_vempty = [&](int s) { return smem_u32(&bars[1 + 3 * C::NS + s]); };
-  auto b_sfull = [&](int b) { return smem_u32(&bars[1 + 4 * C::NS + b]); };
-  auto b_pfull = [&](int b) { return smem_u32(&bars[3 + 4 * C::NS + b]); };
-  auto b_pvdone = [&](int b) { return smem_u32(&bars[5 + 4 * C::NS + b]); };
+  auto b_sfull = [&](int t) { return smem_u32(&bars[1 + 4 * C::NS + t]); };
+  auto b_pfull = [&](int t) { return smem_u32(&bars[3 + 4 * C::NS + t]); };
+  auto b_pvdone = [&](int t) { return smem_u32(&bars[5 + 4 * C::NS + t]); };
   const uint32_t b_drain = smem_u32(&bars[7 + 4 * C::NS]);
-  auto b_xch = [&](int b) { return smem_u32(&bars[8 + 4 * C::NS + b]); };
-  const uint32_t b_ep1 = smem_u32(&bars[10 + 4 * C::NS]);
-  const uint32_t b_ep2 = smem_u32(&bars[11 + 4 * C::NS]);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   // head-major order: the query tiles of one (b, h) run side by side and share its K~, V in
-  // L2; within a head the longest causal tiles go first
+  // L2; within a head the longest causal pairs go first
   const int bh = blockIdx.y;
-  const int qt = p.nq - 1 - blockIdx.x;
+  const int qp = p.npair - 1 - blockIdx.x;
   const int n = p.n;
-  const int T = p.causal ? qt + 1 : (n + C::BN - 1) / C::BN;
+  const int nk = (n + C::BN - 1) / C::BN;
+  // key tiles visited by query tile t = 2 qp + t (tile 1 may lie past n: its rows are
+  // computed on zero-filled queries and never stored)
+  const int T0 = p.causal ? 2 * qp + 1 : nk;
+  const int T1 = p.causal ? 2 * qp + 2 : nk;
   const uint64_t lim = p.limit_ns;
 
   if (tid == 0) {
@@ -110,15 +119,12 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
       mbar_init(b_vfull(s), 1);
       mbar_init(b_vempty(s), 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(b_sfull(b), 1);
-      mbar_init(b_pfull(b), 256);
-      mbar_init(b_pvdone(b), 1);
-      mbar_init(b_xch(b), 256);
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(b_sfull(t), 1);
+      mbar_init(b_pfull(t), 128);
+      mbar_init(b_pvdone(t), 1);
     }
     mbar_init(b_drain, 1);
-    mbar_init(b_ep1, 256);
-    mbar_init(b_ep2, 256);
     abort_set(abort_flag, 0);
     fence_barrier_init();
   }
@@ -131,17 +137,21 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
   tc_fence_after();
   const uint32_t tmem = *tslot;
 
+  if (warp >= 8) regs_dec<C::REG_OTHER>();
+
   if (warp == C::W_PROD) {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
       tma_prefetch(&tm_q);
       tma_prefetch(&tm_k);
       tma_prefetch(&tm_v);
-      mbar_expect_tx(b_q, C::TILE);
-      for (int b = 0; b < C::KB; ++b)
-        tma_load_3d(sbase + C::Q_OFF + b * C::BLK, &tm_q, b_q, 64 * b, qt * C::BM, bh);
+      mbar_expect_tx(b_q, 2 * C::TILE);
+      for (int t = 0; t < 2; ++t)
+        for (int b = 0; b < C::KB; ++b)
+          tma_load_3d(sbase + C::Q_OFF + t * C::TILE + b * C::BLK, &tm_q, b_q, 64 * b,
+                      (2 * qp + t) * C::BM, bh);
       int last_k = -1, last_v = -1;
-      for (int j = 0; j < T; ++j) {
+      for (int j = 0; j < T1; ++j) {
         const int s = j % C::NS;
         const uint32_t ph = (j / C::NS) & 1;
         if (!mbar_wait(b_kempty(s), ph ^ 1, abort_flag, lim)) break;
@@ -169,40 +179,68 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
     }
   } else if (warp == C::W_MMA) {
     // ------------------------------------------------------------------ MMA issuer
+    // issue order per key tile j: PV_0,j, S_0,j+1, PV_1,j, S_1,j+1
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, false, false);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, false, true);
-      bool ok = mbar_wait(b_q, 0, abort_flag, lim);
-      tc_fence_after();
-      for (int j = 0; ok && j <= T; ++j) {
-        if (j < T) {
-          const int s = j % C::NS;
-          if (!(ok = mbar_wait(b_kfull(s), (j / C::NS) & 1, abort_flag, lim))) break;
-          tc_fence_after();
-          const uint32_t d_s = tmem + ((j & 1) ? C::T_S1 : C::T_S0);
-          const uint32_t qa = sbase + C::Q_OFF, kb = sbase + C::K_OFF + s * C::TILE;
+      const uint32_t qa0 = sbase + C::Q_OFF;
+      auto issue_s = [&](int t, int j) {
+        const uint32_t qa = qa0 + t * C::TILE;
+        const uint32_t kb = sbase + C::K_OFF + (j % C::NS) * C::TILE;
+        const uint32_t d_s = tmem + C::T_S0 + 128 * t;
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * C::BLK + (kk & 3) * 32;
-            mma_ss(d_s, sw128_desc(qa + off, 16, 1024), sw128_desc(kb + off, 16, 1024), idesc_s,
-                   kk > 0);
-          }
-          mma_commit(b_sfull(j & 1));
-          mma_commit(b_kempty(s));
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * C::BLK + (kk & 3) * 32;
+          mma_ss(d_s, sw128_desc(qa + off, 16, 1024), sw128_desc(kb + off, 16, 1024), idesc_s,
+                 kk > 0);
         }
-        if (j >= 1) {
-          const int jj = j - 1, s = jj % C::NS, sb = jj & 1;
-          if (!(ok = mbar_wait(b_pfull(sb), (jj >> 1) & 1, abort_flag, lim))) break;
-          if (!(ok = mbar_wait(b_vfull(s), (jj / C::NS) & 1, abort_flag, lim))) break;
-          tc_fence_after();
-          const uint32_t pa = tmem + (sb ? C::T_P1 : C::T_P0);
-          const uint32_t vb = sbase + C::V_OFF + s * C::TILE;
+        mma_commit(b_sfull(t));
+      };
+      auto issue_pv = [&](int t, int j) {
+        const uint32_t pa = tmem + C::T_S0 + 128 * t;
+        const uint32_t vb = sbase + C::V_OFF + (j % C::NS) * C::TILE;
 #pragma unroll
-          for (int kk = 0; kk < C::BN / 16; ++kk)
-            mma_ts(tmem + C::T_O, pa + kk * 8, sw128_desc(vb + kk * 2048, C::BLK, 1024), idesc_pv,
-                   (jj > 0 || kk > 0));
-          mma_commit(b_pvdone(sb));
-          mma_commit(b_vempty(s));
+        for (int kk = 0; kk < C::BN / 16; ++kk)
+          mma_ts(tmem + C::T_O0 + 128 * t, pa + kk * 8, sw128_desc(vb + kk * 2048, C::BLK, 1024),
+                 idesc_pv, (j > 0 || kk > 0));
+        mma_commit(b_pvdone(t));
+      };
+      bool ok = mbar_wait(b_q, 0, abort_flag, lim);
+      if (ok) ok = mbar_wait(b_kfull(0), 0, abort_flag, lim);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0, 0);
+        issue_s(1, 0);
+        mma_commit(b_kempty(0));
+      }
+      for (int j = 0; ok && j < T1; ++j) {
+        const int s = j % C::NS;
+        const bool next0 = j + 1 < T0, next1 = j + 1 < T1;
+        if (!(ok = mbar_wait(b_vfull(s), (j / C::NS) & 1, abort_flag, lim))) break;
+        if (j < T0) {
+          if (!(ok = mbar_wait(b_pfull(0), j & 1, abort_flag, lim))) break;
+          tc_fence_after();
+          issue_pv(0, j);
+        }
+        if (next1) {
+          const int s1 = (j + 1) % C::NS;
+          if (!(ok = mbar_wait(b_kfull(s1), ((j + 1) / C::NS) & 1, abort_flag, lim))) break;
+        }
+        if (next0) {
+          // S_0,j+1 overwrites P_0,j: wait until the product reading it has completed
+          if (!(ok = mbar_wait(b_pvdone(0), j & 1, abort_flag, lim))) break;
+          tc_fence_after();
+          issue_s(0, j + 1);
+        }
+        if (!(ok = mbar_wait(b_pfull(1), j & 1, abort_flag, lim))) break;
+        tc_fence_after();
+        issue_pv(1, j);
+        mma_commit(b_vempty(s));
+        if (next1) {
+          if (!(ok = mbar_wait(b_pvdone(1), j & 1, abort_flag, lim))) break;
+          tc_fence_after();
+          issue_s(1, j + 1);
+          mma_commit(b_kempty((j + 1) % C::NS));
         }
       }
       if (!ok) {
@@ -211,119 +249,102 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
         mbar_drain(b_drain, 0, lim);
       }
     }
-  } else {
+  } else if (warp < 8) {
     // ------------------------------------------------------------------ softmax warps 0-7
-    // warp w reaches TMEM lanes 32 (w % 4) ...; warpgroup `half` takes key columns
-    // 64 half .. 64 half + 63 of each tile and head-dimension columns D/2 half .. of O
-    const int r = tid & 127, half = warp >> 2;
+    // warpgroup t = warp / 4 owns query tile 2 qp + t; warp w reaches TMEM lanes 32 (w % 4)
+    regs_inc<C::REG_SOFTMAX>();
+    const int t = warp >> 2, r = tid & 127;
+    const int qt = 2 * qp + t;
     const int row = qt * C::BM + r;
+    const int Tt = t ? T1 : T0;
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    const uint32_t xch = sbase + C::XCH_OFF;
-    constexpr int OH = D / 2;  // O columns per warpgroup
+    const uint32_t s_col = tmem + lane_base + C::T_S0 + 128 * t;
+    const uint32_t o_col = tmem + lane_base + C::T_O0 + 128 * t;
     float m = -INFINITY, l = 0.f;
     bool ok = true;
-    for (int j = 0; j < T; ++j) {
-      const int sb = j & 1;
-      if (!(ok = mbar_wait_warp(b_sfull(sb), (j >> 1) & 1, abort_flag, lim))) break;
+    for (int j = 0; j < Tt; ++j) {
+      if (!(ok = mbar_wait_warp(b_sfull(t), j & 1, abort_flag, lim))) break;
       tc_fence_after();
-      float x[64];
-      {
-        const uint32_t s_addr = tmem + lane_base + (sb ? C::T_S1 : C::T_S0) + 64 * half;
-        uint32_t r0[32], r1[32];
-        tmem_ld32(s_addr, r0);
-        tmem_ld32(s_addr + 32, r1);
+      float x[128];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t rr[32];
+        tmem_ld32(s_col + 32 * c, rr);
         tmem_wait_ld();
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          x[i] = __uint_as_float(r0[i]);
-          x[32 + i] = __uint_as_float(r1[i]);
-        }
+        for (int i = 0; i < 32; ++i) x[32 * c + i] = __uint_as_float(rr[i]);
       }
-      // raw scores: the scale log2(e)/sqrt(d) > 0 is applied to the row maximum and folded
-      // into the exponent's argument
-      const int key0 = j * C::BN + 64 * half;
-      if (j * C::BN + C::BN > n || (p.causal && j == qt)) {
+      const int key0 = j * C::BN;
+      if (key0 + C::BN > n || (p.causal && j == qt)) {
 #pragma unroll
-        for (int i = 0; i < 64; ++i) {
+        for (int i = 0; i < 128; ++i) {
           const int key = key0 + i;
           if (key >= n || (p.causal && key > row)) x[i] = -INFINITY;
         }
       }
-      float mt = x[0];
+      float mt0 = x[0], mt1 = x[1], mt2 = x[2], mt3 = x[3];
 #pragma unroll
-      for (int i = 1; i < 64; ++i) mt = fmaxf(mt, x[i]);
-      // the other half of the row's maximum
-      st_shared_f32(xch + ((sb * 2 + half) * 128 + r) * 4, mt);
-      mbar_arrive(b_xch(sb));
-      if (!(ok = mbar_wait_warp(b_xch(sb), (j >> 1) & 1, abort_flag, lim))) break;
-      const float mo = ld_shared_f32(xch + ((sb * 2 + (half ^ 1)) * 128 + r) * 4);
-      const float mnew = fmaxf(m, fmaxf(mt, mo) * p.scale_log2);
+      for (int i = 4; i < 128; i += 4) {
+        mt0 = fmaxf(mt0, x[i]);
+        mt1 = fmaxf(mt1, x[i + 1]);
+        mt2 = fmaxf(mt2, x[i + 2]);
+        mt3 = fmaxf(mt3, x[i + 3]);
+      }
+      const float mnew = fmaxf(m, fmaxf(fmaxf(mt0, mt1), fmaxf(mt2, mt3)) * p.scale_log2);
       if (j == 0) {
         m = mnew;
       } else {
-        // both halves of a row take the same decision (same m, same mnew), and warps w and
-        // w + 4 hold the same rows, so the vote agrees across the two warpgroups
         const bool need = mnew > m + 8.f;
         if (__any_sync(0xffffffffu, need)) {
-          // O holds P_0..P_{j-1} V: wait for the last product, then rescale in TMEM
-          if (!(ok = mbar_wait_warp(b_pvdone((j - 1) & 1), ((j - 1) >> 1) & 1, abort_flag, lim)))
-            break;
-          tc_fence_after();
+          // S_t,j was issued after the product of tile j - 1 completed, and its commit
+          // covers that product: O_t is final for tiles < j and can be rescaled in place
           const float alpha = need ? ex2(m - mnew) : 1.f;
           if (need) {
             l *= alpha;
             m = mnew;
           }
 #pragma unroll
-          for (int c = 0; c < OH / 32; ++c) {
+          for (int c = 0; c < D / 32; ++c) {
             uint32_t rr[32];
-            const uint32_t oa = tmem + lane_base + C::T_O + OH * half + 32 * c;
-            tmem_ld32(oa, rr);
+            tmem_ld32(o_col + 32 * c, rr);
             tmem_wait_ld();
 #pragma unroll
             for (int i = 0; i < 32; ++i) rr[i] = __float_as_uint(__uint_as_float(rr[i]) * alpha);
-            tmem_st32(oa, rr);
+            tmem_st32(o_col + 32 * c, rr);
           }
-          tmem_wait_st();
         }
       }
-      if (j >= 2) {  // P buffer sb was read by the product of tile j - 2
-        if (!(ok = mbar_wait_warp(b_pvdone(sb), ((j - 2) >> 1) & 1, abort_flag, lim))) break;
-        tc_fence_after();
-      }
-      float psum = 0.f;
-      uint32_t pk[32];
+      float ps0 = 0.f, ps1 = 0.f;
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        const float p0 = ex2(fmaf(x[2 * i], p.scale_log2, -m));
-        const float p1 = ex2(fmaf(x[2 * i + 1], p.scale_log2, -m));
-        psum += p0 + p1;
-        pk[i] = pack_bf16x2(p0, p1);
+      for (int c = 0; c < 4; ++c) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float p0 = ex2(fmaf(x[32 * c + 2 * i], p.scale_log2, -m));
+          const float p1 = ex2(fmaf(x[32 * c + 2 * i + 1], p.scale_log2, -m));
+          ps0 += p0;
+          ps1 += p1;
+          pk[i] = pack_bf16x2(p0, p1);
+        }
+        tmem_st16(s_col + 16 * c, pk);
       }
-      tmem_st32(tmem + lane_base + (sb ? C::T_P1 : C::T_P0) + 32 * half, pk);
-      l += psum;
+      l += ps0 + ps1;
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(b_pfull(sb));
+      mbar_arrive(b_pfull(t));
     }
-    // ---- epilogue: each warpgroup finishes its D/2 columns of O
+    // ---- epilogue: one full row of O per thread
     float sq = 0.f, dl = 0.f;
-    if (ok) ok = mbar_wait_warp(b_pvdone((T - 1) & 1), ((T - 1) >> 1) & 1, abort_flag, lim);
-    st_shared_f32(sbase + C::EPL_OFF + (half * 128 + r) * 4, l);
-    mbar_arrive(b_ep1);
-    const bool ok1 = mbar_wait_warp(b_ep1, 0, abort_flag, lim);
+    if (ok) ok = mbar_wait_warp(b_pvdone(t), (Tt - 1) & 1, abort_flag, lim);
     const bool vrow = row < n;
-    float l_row = 1.f;
-    if (ok && ok1) {
+    if (ok) {
       tc_fence_after();
-      l_row = ld_shared_f32(sbase + C::EPL_OFF + r * 4) +
-              ld_shared_f32(sbase + C::EPL_OFF + (128 + r) * 4);
-      const float inv_l = 1.f / l_row;
-      const size_t ro = ((size_t)bh * n + row) * D + OH * half;
-#pragma unroll
-      for (int c = 0; c < OH / 32; ++c) {
+      const float inv_l = 1.f / l;
+      const size_t ro = ((size_t)bh * n + row) * D;
+#pragma unroll 1
+      for (int c = 0; c < D / 32; ++c) {
         uint32_t rr[32];
-        tmem_ld32(tmem + lane_base + C::T_O + OH * half + 32 * c, rr);
+        tmem_ld32(o_col + 32 * c, rr);
         tmem_wait_ld();
         if (vrow) {
           float o[32];
@@ -356,25 +377,16 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
           }
         }
       }
+      if (vrow) {
+        p.lse[(size_t)bh * n + row] = (m + log2f(l)) * kLn2;
+        if (p.E) p.delta[(size_t)bh * n + row] = dl;
+      }
     }
-    // combine <l, O> of the two halves and the per-warp sums of l^2
-    if (half == 1) st_shared_f32(sbase + C::EPD_OFF + r * 4, dl);
+    // per-warp partial of 1/2 sum l^2 (fixed order: deterministic)
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
-    if (lane == 0) st_shared_f32(red + warp * 4, sq);
-    mbar_arrive(b_ep2);
-    const bool ok2 = mbar_wait_warp(b_ep2, 0, abort_flag, lim);
-    if (ok && ok1 && ok2) {
-      if (half == 0 && vrow) {
-        p.lse[(size_t)bh * n + row] = (m + log2f(l_row)) * kLn2;
-        if (p.E) p.delta[(size_t)bh * n + row] = dl + ld_shared_f32(sbase + C::EPD_OFF + r * 4);
-      }
-      if (p.E && tid == 0) {
-        double t = 0.0;
-        for (int w = 0; w < 8; ++w) t += (double)ld_shared_f32(red + w * 4);
-        p.loss_part[(size_t)blockIdx.y * gridDim.x + blockIdx.x] = 0.5 * t;
-      }
-    }
+    if (p.E && ok && lane == 0 && qt < p.nq)
+      p.loss_part[((size_t)bh * p.nq + qt) * C::LOSS_PARTS + (warp & 3)] = 0.5 * (double)sq;
   }
   tc_fence_before();
   __syncthreads();

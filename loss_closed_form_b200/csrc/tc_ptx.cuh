@@ -131,6 +131,18 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
 // ---------------------------------------------------------------------------------------
 // tcgen05
 // ---------------------------------------------------------------------------------------
+// Move registers between warpgroups (every thread of the warpgroup executes it; the new
+// count is a multiple of 8 in [24, 256]).  Increases draw on the registers the CTA was
+// launched with, which decreases by other warpgroups return.
+template <int N>
+__device__ __forceinline__ void regs_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void regs_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 // Allocate `ncols` TMEM columns (power of 2, >= 32); whole warp; address written to smem.
 __device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {
   asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem),
