@@ -196,6 +196,15 @@ T* at(void* ws, size_t off) {
   return reinterpret_cast<T*>(static_cast<char*>(ws) + off);
 }
 
+// SM count of the current device (persistent grids take one CTA per SM).
+int num_sms() {
+  int dev = 0, v = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0)
+    return 148;
+  return v;
+}
+
 ra_status launch_status() {
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? RA_OK : RA_ERR_CUDA;
@@ -336,32 +345,31 @@ ra_status tc_project(const ra_problem* p, const Layout& L, void* ws, cudaStream_
     ra::simt::rope_table_kernel<<<(total + 255) / 256, 256, 0, st>>>(tab, p->pos, n, half,
                                                                      p->rope_base);
   }
-  CUtensorMap a1, a2, a3, w1, w2, w3;
+  CUtensorMap a1, a2, a3, w1, w2, w3, o1, o2, o3;
   if (!map_bf16_3d(&a1, p->A1, D, n, BH, C::BM) || !map_bf16_3d(&a2, p->A2, D, n, BH, C::BM) ||
       !map_bf16_3d(&a3, p->A3, D, n, BH, C::BM) || !map_bf16_3d(&w1, p->WQ, D, D, p->H, D) ||
-      !map_bf16_3d(&w2, p->WK, D, D, p->H, D) || !map_bf16_3d(&w3, p->WV, D, D, p->H, D))
+      !map_bf16_3d(&w2, p->WK, D, D, p->H, D) || !map_bf16_3d(&w3, p->WV, D, D, p->H, D) ||
+      !map_bf16_3d(&o1, at<void>(ws, L.qt), D, n, BH, C::BM) ||
+      !map_bf16_3d(&o2, at<void>(ws, L.kt), D, n, BH, C::BM) ||
+      !map_bf16_3d(&o3, at<void>(ws, L.v), D, n, BH, C::BM))
     return RA_ERR_CUDA;
   ProjParams pp;
   pp.tab = tab;
-  pp.out[0] = at<__nv_bfloat16>(ws, L.qt);
-  pp.out[1] = at<__nv_bfloat16>(ws, L.kt);
-  pp.out[2] = at<__nv_bfloat16>(ws, L.v);
   pp.n = n;
   pp.B = p->B;
   pp.H = p->H;
   pp.nrt = (n + C::BM - 1) / C::BM;
-  // persistent CTAs over the 128-row tiles of one (z, h): about two waves of 148 CTAs
-  const long tiles = (long)p->B * pp.nrt;
-  long chunks = (2 * 148 + 3 * p->H - 1) / (3 * p->H);
-  chunks = chunks < 1 ? 1 : (chunks > tiles ? tiles : chunks);
-  pp.tiles_per_cta = (int)((tiles + chunks - 1) / chunks);
-  chunks = (tiles + pp.tiles_per_cta - 1) / pp.tiles_per_cta;
+  // persistent CTAs, one per SM, over the (row tile, z, head) tiles
+  pp.tiles = (long long)p->B * pp.nrt * 3 * p->H;
+  const long long sms = num_sms();
+  const long long ctas = pp.tiles < sms ? pp.tiles : sms;
+  pp.tiles_per_cta = (pp.tiles + ctas - 1) / ctas;
+  const long long grid = (pp.tiles + pp.tiles_per_cta - 1) / pp.tiles_per_cta;
   pp.limit_ns = wait_limit_ns();
   auto k = proj_rope_tc_kernel<D>;
   cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_ALLOC);
-  dim3 grid((unsigned)chunks, p->H, 3);
   Launch l(K_PROJ_TC, st);
-  k<<<grid, C::THREADS, C::SMEM_ALLOC, st>>>(a1, a2, a3, w1, w2, w3, pp);
+  k<<<(unsigned)grid, C::THREADS, C::SMEM_ALLOC, st>>>(a1, a2, a3, w1, w2, w3, o1, o2, o3, pp);
   return launch_status();
 }
 

@@ -18,43 +18,54 @@ namespace tc {
 // ---------------------------------------------------------------------------------------
 // projections + RoPE
 // ---------------------------------------------------------------------------------------
+// Persistent kernel over 128-row tiles ordered (row tile, z, head) with the head fastest, so
+// a CTA keeps one row tile's RoPE angles (cos, sin) in registers while it runs through the
+// heads.  Per tile: TMA loads A_z[b, h] rows and W_z[h]; one tcgen05 product into a
+// double-buffered TMEM accumulator; the epilogue warps rotate, round to bf16 and write a
+// 128-byte-swizzled staging tile that a TMA store sends to global memory (the staging is
+// double-buffered, so the store of one tile overlaps the next tile's epilogue).
 template <int D>
 struct ProjCfg {
   static constexpr int BM = 128;
   static constexpr int KB = D / 64;
-  static constexpr int NS = 4;               // A-tile stages
+  static constexpr int NS = 2;               // (A, W) load stages
   static constexpr int ATILE = BM * D * 2;
   static constexpr int WTILE = D * D * 2;
   static constexpr int ABLK = BM * 128;      // [128 rows][64 cols] block
   static constexpr int WBLK = D * 128;       // [D rows][64 cols] block
-  static constexpr int W_OFF = 0;
-  static constexpr int A_OFF = WTILE;
-  static constexpr int BAR_OFF = A_OFF + NS * ATILE;
-  // w_full, a_full[NS], a_empty[NS], acc_full[2], acc_empty[2], drain
-  static constexpr int NBAR = 1 + 2 * NS + 4 + 1;
+  static constexpr int OTILE = BM * D * 2;   // bf16 output staging tile
+  static constexpr int A_OFF = 0;
+  static constexpr int W_OFF = A_OFF + NS * ATILE;
+  static constexpr int O_OFF = W_OFF + NS * WTILE;
+  static constexpr int BAR_OFF = O_OFF + 2 * OTILE;
+  // ld_full[NS], ld_empty[NS], acc_full[2], acc_empty[2], o_full[2], o_free[2], drain
+  static constexpr int NBAR = 2 * NS + 8 + 1;
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
   static constexpr int SMEM_ALLOC = MISC_OFF + 16 + 1024;
-  static constexpr int THREADS = 192;        // warps 0-3 epilogue, 4 TMA, 5 MMA
+  // warps 0-7 epilogue (warp w: TMEM lanes 32 (w % 4), columns D/2 (w / 4) ..), 8 TMA
+  // loads, 9 MMA, 10 TMA stores
+  static constexpr int THREADS = 352;
+  static constexpr int W_LOAD = 8, W_MMA = 9, W_STORE = 10;
+  static constexpr int CPT = D / 2;          // output columns per epilogue thread
   static constexpr uint32_t T_COLS = 2 * D;  // double-buffered accumulator
+  static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
 };
 
 struct ProjParams {
   const float2* tab;       // [n][d/2] (cos, sin)
-  __nv_bfloat16* out[3];   // Q~, K~, V: [BH][n][d]
   int n, B, H, nrt;        // nrt = 128-row tiles per instance
-  int tiles_per_cta;
+  long long tiles;         // B * nrt * 3 * H
+  long long tiles_per_cta;
   unsigned long long limit_ns;
 };
 
-// grid (chunks, H, 3): the CTA (c, h, z) projects tiles t = b * nrt + rt in
-// [c * tiles_per_cta, ...) of head h with W_z[h] loaded once; z = 0 (Q, rotated),
-// 1 (K, rotated), 2 (V).
 template <int D>
 __global__ void __launch_bounds__(ProjCfg<D>::THREADS, 1)
 proj_rope_tc_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_constant__ CUtensorMap tm_a2,
                     const __grid_constant__ CUtensorMap tm_a3, const __grid_constant__ CUtensorMap tm_w1,
                     const __grid_constant__ CUtensorMap tm_w2, const __grid_constant__ CUtensorMap tm_w3,
-                    const ProjParams p) {
+                    const __grid_constant__ CUtensorMap tm_o1, const __grid_constant__ CUtensorMap tm_o2,
+                    const __grid_constant__ CUtensorMap tm_o3, const ProjParams p) {
   using C = ProjCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -63,34 +74,43 @@ proj_rope_tc_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_cons
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
   uint32_t* tslot = reinterpret_cast<uint32_t*>(smem + C::MISC_OFF);
   const uint32_t abort_flag = smem_u32(smem + C::MISC_OFF + 4);
-  const uint32_t b_w = smem_u32(&bars[0]);
-  auto b_afull = [&](int s) { return smem_u32(&bars[1 + s]); };
-  auto b_aempty = [&](int s) { return smem_u32(&bars[1 + C::NS + s]); };
-  auto b_accfull = [&](int b) { return smem_u32(&bars[1 + 2 * C::NS + b]); };
-  auto b_accempty = [&](int b) { return smem_u32(&bars[3 + 2 * C::NS + b]); };
-  const uint32_t b_drain = smem_u32(&bars[5 + 2 * C::NS]);
+  auto b_ldfull = [&](int s) { return smem_u32(&bars[s]); };
+  auto b_ldempty = [&](int s) { return smem_u32(&bars[C::NS + s]); };
+  auto b_accfull = [&](int b) { return smem_u32(&bars[2 * C::NS + b]); };
+  auto b_accempty = [&](int b) { return smem_u32(&bars[2 * C::NS + 2 + b]); };
+  auto b_ofull = [&](int b) { return smem_u32(&bars[2 * C::NS + 4 + b]); };
+  auto b_ofree = [&](int b) { return smem_u32(&bars[2 * C::NS + 6 + b]); };
+  const uint32_t b_drain = smem_u32(&bars[2 * C::NS + 8]);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int h = blockIdx.y, z = blockIdx.z;
-  const CUtensorMap* tma = z == 0 ? &tm_a1 : z == 1 ? &tm_a2 : &tm_a3;
-  const CUtensorMap* tmw = z == 0 ? &tm_w1 : z == 1 ? &tm_w2 : &tm_w3;
-  const int t0 = blockIdx.x * p.tiles_per_cta;
-  const int NT = min(p.tiles_per_cta, p.B * p.nrt - t0);
+  const long long t0 = (long long)blockIdx.x * p.tiles_per_cta;
+  const int NT = (int)min(p.tiles_per_cta, p.tiles - t0);
   const uint64_t lim = p.limit_ns;
+  // tile index -> (b, row tile, z, h): head fastest, then z, then row tile
+  auto decode = [&](int t, int& b, int& rt, int& z, int& h) {
+    long long q = t0 + t;
+    h = (int)(q % p.H);
+    q /= p.H;
+    z = (int)(q % 3);
+    q /= 3;
+    rt = (int)(q % p.nrt);
+    b = (int)(q / p.nrt);
+  };
   if (tid == 0) {
-    mbar_init(b_w, 1);
     for (int s = 0; s < C::NS; ++s) {
-      mbar_init(b_afull(s), 1);
-      mbar_init(b_aempty(s), 1);
+      mbar_init(b_ldfull(s), 1);
+      mbar_init(b_ldempty(s), 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(b_accfull(b), 1);
-      mbar_init(b_accempty(b), 128);
+      mbar_init(b_accempty(b), 256);
+      mbar_init(b_ofull(b), 256);
+      mbar_init(b_ofree(b), 1);
     }
     mbar_init(b_drain, 1);
     abort_set(abort_flag, 0);
     fence_barrier_init();
   }
-  if (warp == 5) {
+  if (warp == C::W_MMA) {
     tmem_alloc(smem_u32(tslot), C::T_COLS);
     tmem_relinquish();
   }
@@ -98,97 +118,136 @@ proj_rope_tc_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_cons
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tslot;
-  if (warp == 4) {
-    // ------------------------------------------------------------------ TMA producer
+  if (warp == C::W_LOAD) {
+    // ------------------------------------------------------------------ TMA loads
     if (lane == 0) {
-      mbar_expect_tx(b_w, C::WTILE);
-      for (int b = 0; b < C::KB; ++b)
-        tma_load_3d(sbase + C::W_OFF + b * C::WBLK, tmw, b_w, 64 * b, 0, h);
+      tma_prefetch(&tm_a1);
+      tma_prefetch(&tm_a2);
+      tma_prefetch(&tm_a3);
       int last = -1;
       for (int t = 0; t < NT; ++t) {
         const int s = t % C::NS;
-        if (!mbar_wait(b_aempty(s), ((t / C::NS) & 1) ^ 1, abort_flag, lim)) break;
-        const int tt = t0 + t, b = tt / p.nrt, rt = tt - b * p.nrt;
-        mbar_expect_tx(b_afull(s), C::ATILE);
-        for (int kb = 0; kb < C::KB; ++kb)
-          tma_load_3d(sbase + C::A_OFF + s * C::ATILE + kb * C::ABLK, tma, b_afull(s), 64 * kb,
+        if (!mbar_wait(b_ldempty(s), ((t / C::NS) & 1) ^ 1, abort_flag, lim)) break;
+        int b, rt, z, h;
+        decode(t, b, rt, z, h);
+        const CUtensorMap* tma = z == 0 ? &tm_a1 : z == 1 ? &tm_a2 : &tm_a3;
+        const CUtensorMap* tmw = z == 0 ? &tm_w1 : z == 1 ? &tm_w2 : &tm_w3;
+        mbar_expect_tx(b_ldfull(s), C::ATILE + C::WTILE);
+        for (int kb = 0; kb < C::KB; ++kb) {
+          tma_load_3d(sbase + C::A_OFF + s * C::ATILE + kb * C::ABLK, tma, b_ldfull(s), 64 * kb,
                       rt * C::BM, b * p.H + h);
+          tma_load_3d(sbase + C::W_OFF + s * C::WTILE + kb * C::WBLK, tmw, b_ldfull(s), 64 * kb,
+                      0, h);
+        }
         last = t;
       }
       if (abort_get(abort_flag)) {
-        mbar_drain(b_w, 0, lim);
         for (int t = (last - C::NS + 1 > 0 ? last - C::NS + 1 : 0); t <= last; ++t)
-          mbar_drain(b_afull(t % C::NS), (t / C::NS) & 1, lim);
+          mbar_drain(b_ldfull(t % C::NS), (t / C::NS) & 1, lim);
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == C::W_MMA) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_bf16_f32(128, D, false, true);
-      bool ok = mbar_wait(b_w, 0, abort_flag, lim);
+      bool ok = true;
       for (int t = 0; ok && t < NT; ++t) {
         const int s = t % C::NS, ab = t & 1;
-        if (!(ok = mbar_wait(b_afull(s), (t / C::NS) & 1, abort_flag, lim))) break;
+        if (!(ok = mbar_wait(b_ldfull(s), (t / C::NS) & 1, abort_flag, lim))) break;
         if (!(ok = mbar_wait(b_accempty(ab), ((t >> 1) & 1) ^ 1, abort_flag, lim))) break;
         tc_fence_after();
         const uint32_t a = sbase + C::A_OFF + s * C::ATILE;
+        const uint32_t w = sbase + C::W_OFF + s * C::WTILE;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
           mma_ss(tmem + ab * D, sw128_desc(a + (kk >> 2) * C::ABLK + (kk & 3) * 32, 16, 1024),
-                 sw128_desc(sbase + C::W_OFF + kk * 2048, C::WBLK, 1024), idesc, kk > 0);
+                 sw128_desc(w + kk * 2048, C::WBLK, 1024), idesc, kk > 0);
         mma_commit(b_accfull(ab));
-        mma_commit(b_aempty(s));
+        mma_commit(b_ldempty(s));
       }
       if (!ok) {
         mma_commit(b_drain);
         mbar_drain(b_drain, 0, lim);
       }
     }
-  } else {
-    // ------------------------------------------------------------------ epilogue (warps 0-3)
-    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-    __nv_bfloat16* out_base = p.out[z];
+  } else if (warp == C::W_STORE) {
+    // ------------------------------------------------------------------ TMA stores
+    if (lane == 0) {
+      for (int t = 0; t < NT; ++t) {
+        const int ob = t & 1;
+        if (!mbar_wait(b_ofull(ob), (t >> 1) & 1, abort_flag, lim)) break;
+        int b, rt, z, h;
+        decode(t, b, rt, z, h);
+        const CUtensorMap* tmo = z == 0 ? &tm_o1 : z == 1 ? &tm_o2 : &tm_o3;
+        for (int kb = 0; kb < C::KB; ++kb)
+          tma_store_3d(tmo, sbase + C::O_OFF + ob * C::OTILE + kb * C::ABLK, 64 * kb, rt * C::BM,
+                       b * p.H + h);
+        bulk_commit();
+        bulk_wait_read0();
+        mbar_arrive(b_ofree(ob));
+      }
+      bulk_wait0();  // the stores have landed before the CTA leaves
+    }
+  } else if (warp < 8) {
+    // ------------------------------------------------------------------ epilogue (warps 0-7)
+    const int rl = 32 * (warp & 3) + lane;           // row within the tile = TMEM lane
+    const int c0 = C::CPT * (warp >> 2);             // first output column of this thread
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    float2 cs[C::CPT / 2];                            // (cos, sin) of this row's pairs
+    int key = -1;                                     // row tile the angles belong to
     for (int t = 0; t < NT; ++t) {
       const int ab = t & 1;
+      int b, rt, z, h;
+      decode(t, b, rt, z, h);
+      const int row = rt * C::BM + rl;
+      if (z < 2 && rt != key) {
+        key = rt;
+        const float4* tr = reinterpret_cast<const float4*>(p.tab + (size_t)(row < p.n ? row : 0) * (D / 2) + c0 / 2);
+#pragma unroll
+        for (int k = 0; k < C::CPT / 4; ++k) {
+          const float4 v = tr[k];
+          cs[2 * k] = make_float2(v.x, v.y);
+          cs[2 * k + 1] = make_float2(v.z, v.w);
+        }
+      }
       if (!mbar_wait_warp(b_accfull(ab), (t >> 1) & 1, abort_flag, lim)) break;
       tc_fence_after();
-      const int tt = t0 + t, b = tt / p.nrt, rt = tt - b * p.nrt;
-      const int row = rt * C::BM + tid;
-      const bool vrow = row < p.n;
-      uint32_t r[D];
+      uint32_t r[C::CPT];
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c)
-        tmem_ld32(tmem + lane_base + ab * D + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&r[32 * c]));
+      for (int c = 0; c < C::CPT / 32; ++c)
+        tmem_ld32(tmem + lane_base + ab * D + c0 + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&r[32 * c]));
       tmem_wait_ld();
       tc_fence_before();
       mbar_arrive(b_accempty(ab));
-      if (vrow) {
-        __nv_bfloat16* out = out_base + ((size_t)(b * p.H + h) * p.n + row) * D;
-        const float4* tr = reinterpret_cast<const float4*>(p.tab + (size_t)row * (D / 2));
+      // staging buffer ob is free once the store of tile t - 2 has read it
+      const int ob = t & 1;
+      if (t >= 2 && !mbar_wait_warp(b_ofree(ob), ((t - 2) >> 1) & 1, abort_flag, lim)) break;
+      const uint32_t ost = sbase + C::O_OFF + ob * C::OTILE;
 #pragma unroll
-        for (int c = 0; c < D / 8; ++c) {  // 8 columns = 4 pairs = one 16-byte store
-          uint32_t w[4];
+      for (int c = 0; c < C::CPT / 8; ++c) {  // 8 columns = 4 pairs = one 16-byte chunk
+        uint32_t w[4];
 #pragma unroll
-          for (int k2 = 0; k2 < 2; ++k2) {
-            float x0 = __uint_as_float(r[8 * c + 4 * k2]), x1 = __uint_as_float(r[8 * c + 4 * k2 + 1]);
-            float x2 = __uint_as_float(r[8 * c + 4 * k2 + 2]), x3 = __uint_as_float(r[8 * c + 4 * k2 + 3]);
-            if (z < 2) {
-              const float4 cs = tr[2 * c + k2];  // (cos, sin) of two consecutive pairs
-              const float y0 = x0 * cs.x - x1 * cs.y, y1 = x0 * cs.y + x1 * cs.x;
-              const float y2 = x2 * cs.z - x3 * cs.w, y3 = x2 * cs.w + x3 * cs.z;
-              x0 = y0; x1 = y1; x2 = y2; x3 = y3;
-            }
-            w[2 * k2] = pack_bf16x2(x0, x1);
-            w[2 * k2 + 1] = pack_bf16x2(x2, x3);
+        for (int k2 = 0; k2 < 4; ++k2) {
+          float x0 = __uint_as_float(r[8 * c + 2 * k2]), x1 = __uint_as_float(r[8 * c + 2 * k2 + 1]);
+          if (z < 2) {
+            const float2 a = cs[4 * c + k2];
+            const float y0 = x0 * a.x - x1 * a.y, y1 = x0 * a.y + x1 * a.x;
+            x0 = y0;
+            x1 = y1;
           }
-          reinterpret_cast<uint4*>(out)[c] = make_uint4(w[0], w[1], w[2], w[3]);
+          w[k2] = pack_bf16x2(x0, x1);
         }
+        const int col = c0 + 8 * c;
+        st_shared_v4(ost + (col >> 6) * C::ABLK + sw128_offset(rl, (col & 63) >> 3), w[0], w[1],
+                     w[2], w[3]);
       }
+      fence_proxy_async_smem();
+      mbar_arrive(b_ofull(ob));
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == C::W_MMA) {
     tc_fence_after();
     tmem_dealloc(tmem, C::T_COLS);
   }
