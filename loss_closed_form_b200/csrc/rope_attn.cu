@@ -325,7 +325,7 @@ ra_status simt_fwd(const ra_problem* p, void* O, float* lse, float* loss, void* 
   }
   if (loss) {
     Launch l(K_LOSS, st);
-    loss_finalize_kernel<<<1, 256, 0, st>>>(at<double>(ws, L.loss_part), L.nparts_fwd, loss);
+    loss_finalize_kernel<<<1, 1024, 0, st>>>(at<double>(ws, L.loss_part), L.nparts_fwd, loss);
   }
   return launch_status();
 }
@@ -380,11 +380,10 @@ ra_status tc_weight_grads(const ra_problem* p, const Layout& L, float* dWQ, floa
   using C = DwCfg<D>;
   const int n = p->n, BH = p->B * p->H, half = D / 2;
   {
-    const long long pairs = (long long)BH * n * half;
+    const long long quads = (long long)BH * n * (half / 4);
     Launch l(K_DQ_UNROT, st);
-    dq_unrotate_kernel<<<(unsigned)((pairs + 255) / 256), 256, 0, st>>>(
-        at<float2>(ws, L.dqt), at<float2>(ws, L.rope), at<__nv_bfloat162>(ws, L.dq16), pairs, n,
-        half);
+    dq_unrotate_kernel<<<(unsigned)((quads + 255) / 256), 256, 0, st>>>(
+        at<float4>(ws, L.dqt), at<float4>(ws, L.rope), at<uint4>(ws, L.dq16), quads, n, half);
   }
   CUtensorMap a1, a2, a3, x1, x2, x3;
   if (!map_bf16_3d(&a1, p->A1, D, n, BH, C::BR) || !map_bf16_3d(&a2, p->A2, D, n, BH, C::BR) ||
@@ -461,7 +460,7 @@ ra_status tc_fwd(const ra_problem* p, void* O, float* lse, float* loss, void* ws
   if (s != RA_OK) return s;
   if (loss) {
     Launch l(K_LOSS, st);
-    ra::simt::loss_finalize_kernel<<<1, 256, 0, st>>>(at<double>(ws, L.loss_part), L.nparts_fwd,
+    ra::simt::loss_finalize_kernel<<<1, 1024, 0, st>>>(at<double>(ws, L.loss_part), L.nparts_fwd,
                                                       loss);
   }
   return launch_status();
@@ -548,7 +547,7 @@ ra_status simt_bwd(const ra_problem* p, const void* O, const float* lse, float* 
   }
   if (loss) {
     Launch l(K_LOSS, st);
-    loss_finalize_kernel<<<1, 256, 0, st>>>(at<double>(ws, L.loss_part),
+    loss_finalize_kernel<<<1, 1024, 0, st>>>(at<double>(ws, L.loss_part),
                                             holds ? L.nparts_fwd : L.nparts_pre, loss);
   }
   return launch_status();
@@ -579,7 +578,7 @@ ra_status tc_bwd(const ra_problem* p, const void* O, const float* lse, float* lo
   if (s != RA_OK) return s;
   if (loss) {
     Launch l(K_LOSS, st);
-    ra::simt::loss_finalize_kernel<<<1, 256, 0, st>>>(at<double>(ws, L.loss_part),
+    ra::simt::loss_finalize_kernel<<<1, 1024, 0, st>>>(at<double>(ws, L.loss_part),
                                                       holds ? L.nparts_fwd : L.nparts_pre, loss);
   }
   return launch_status();

@@ -437,10 +437,20 @@ __global__ void dw_reduce_kernel(const float* __restrict__ part, float* __restri
 // loss = sum of the partials in a fixed order (fp64), one block of 256 threads.
 __global__ void loss_finalize_kernel(const double* __restrict__ part, int count,
                                      float* __restrict__ loss) {
-  __shared__ double red[256];
-  double s = 0.0;
-  for (int i = threadIdx.x; i < count; i += blockDim.x) s += part[i];
-  red[threadIdx.x] = s;
+  // fixed summation order for a given count and block size (deterministic); four
+  // independent partial sums per thread keep the loads in flight
+  __shared__ double red[1024];
+  double s0 = 0.0, s1 = 0.0, s2 = 0.0, s3 = 0.0;
+  const int stride = blockDim.x;
+  int i = threadIdx.x;
+  for (; i + 3 * stride < count; i += 4 * stride) {
+    s0 += part[i];
+    s1 += part[i + stride];
+    s2 += part[i + 2 * stride];
+    s3 += part[i + 3 * stride];
+  }
+  for (; i < count; i += stride) s0 += part[i];
+  red[threadIdx.x] = (s0 + s1) + (s2 + s3);
   __syncthreads();
   for (int w = blockDim.x / 2; w > 0; w >>= 1) {
     if ((int)threadIdx.x < w) red[threadIdx.x] += red[threadIdx.x + w];

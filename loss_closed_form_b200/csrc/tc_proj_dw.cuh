@@ -254,19 +254,26 @@ proj_rope_tc_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_cons
 }
 
 // ---------------------------------------------------------------------------------------
-// dQ = rot^-1(dQ~): fp32 in, bf16 out; one thread per pair.
+// dQ = rot^-1(dQ~): fp32 in, bf16 out; one thread per four pairs (d/2 is a multiple of 4,
+// so the four pairs share a row): two 16-byte loads of dQ~ and of (cos, sin), one 16-byte
+// store.
 // ---------------------------------------------------------------------------------------
-__global__ void dq_unrotate_kernel(const float2* __restrict__ dqt, const float2* __restrict__ tab,
-                                   __nv_bfloat162* __restrict__ dq, long long pairs, int n,
-                                   int half) {
+__global__ void dq_unrotate_kernel(const float4* __restrict__ dqt, const float4* __restrict__ tab,
+                                   uint4* __restrict__ dq, long long quads, int n, int half) {
   const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  if (idx >= pairs) return;
-  const long long row = idx / half;
-  const int k = (int)(idx - row * half);
+  if (idx >= quads) return;
+  const int qpr = half / 4;  // quads per row
+  const long long row = idx / qpr;
+  const int k = (int)(idx - row * qpr);
   const int i = (int)(row % n);
-  const float2 y = dqt[idx];
-  const float2 cs = tab[(size_t)i * half + k];
-  dq[idx] = __floats2bfloat162_rn(y.x * cs.x + y.y * cs.y, -y.x * cs.y + y.y * cs.x);
+  const float4 y0 = dqt[2 * idx], y1 = dqt[2 * idx + 1];
+  const float4* tr = tab + ((size_t)i * half) / 2 + 2 * k;
+  const float4 c0 = tr[0], c1 = tr[1];
+  auto rot = [](float x, float y, float c, float sn) {
+    return pack_bf16x2(x * c + y * sn, -x * sn + y * c);
+  };
+  dq[idx] = make_uint4(rot(y0.x, y0.y, c0.x, c0.y), rot(y0.z, y0.w, c0.z, c0.w),
+                       rot(y1.x, y1.y, c1.x, c1.y), rot(y1.z, y1.w, c1.z, c1.w));
 }
 
 // ---------------------------------------------------------------------------------------
