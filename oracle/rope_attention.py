@@ -118,7 +118,12 @@ def instance_forward_backward(A1, A2, A3, E, WQ, WK, WV, pos, causal: bool, base
 
     Inputs are [n][d] (A1, A2, A3, E) and [d][d] (WQ, WK, WV).  Returns O, lse, loss and,
     with ``want_grad``, dQt, dKt, dV (gradients w.r.t. the rotated Q~, K~ and V),
-    dQ, dK (un-rotated) and dWQ, dWK, dWV.
+    dQ, dK (un-rotated), dWQ, dWK, dWV and the input gradients dA1, dA2, dA3.
+
+    The weight gradients are the ones the problem of "RoPE Attention kan bijna lineair
+    worden getraind" (Probleemdefinitie) asks for.  The input gradients follow from the same
+    chain rule through Q = A1 WQ, K = A2 WK, V = A3 WV: dA1 = dQ WQ^T, dA2 = dK WK^T,
+    dA3 = dV WV^T (they let layers be stacked; the page itself stops at the weights).
     """
     n, d = np.shape(A1)
     c = 1.0 / math.sqrt(d)
@@ -155,7 +160,10 @@ def instance_forward_backward(A1, A2, A3, E, WQ, WK, WV, pos, causal: bool, base
         out.update(dQt=dQt, dKt=dKt, dV=dV, dQ=dQ, dK=dK,
                    dWQ=np.asarray(A1, F64).T @ dQ,
                    dWK=np.asarray(A2, F64).T @ dK,
-                   dWV=np.asarray(A3, F64).T @ dV)
+                   dWV=np.asarray(A3, F64).T @ dV,
+                   dA1=dQ @ np.asarray(WQ, F64).T,
+                   dA2=dK @ np.asarray(WK, F64).T,
+                   dA3=dV @ np.asarray(WV, F64).T)
     return out
 
 
@@ -175,14 +183,16 @@ def forward_backward(inp: Dict[str, np.ndarray], causal: bool, base: float,
                      want_grad: bool = True) -> Dict[str, np.ndarray]:
     """All (b, h) instances of a batch; ``heads`` restricts the work to some heads.
 
-    Returns O [B][H][n][d], lse [B][H][n], loss (sum over the instances computed) and
-    dWQ, dWK, dWV [H][d][d] (summed over b).  Entries of heads not computed are NaN.
+    Returns O [B][H][n][d], lse [B][H][n], loss (sum over the instances computed),
+    dWQ, dWK, dWV [H][d][d] (summed over b) and, per instance, dQt, dKt, dV, dA1, dA2, dA3
+    [B][H][n][d].  Entries of heads not computed are NaN.
     """
     B, H, n, d = inp["A1"].shape
     O = np.full((B, H, n, d), np.nan)
     lse = np.full((B, H, n), np.nan)
     dW = {k: np.full((H, d, d), np.nan) for k in ("dWQ", "dWK", "dWV")}
-    extra = {k: np.full((B, H, n, d), np.nan) for k in ("dQt", "dKt", "dV")} if want_grad else {}
+    extra = ({k: np.full((B, H, n, d), np.nan) for k in ("dQt", "dKt", "dV", "dA1", "dA2", "dA3")}
+             if want_grad else {})
     loss = 0.0
     for h in _heads(inp, heads):
         if want_grad:

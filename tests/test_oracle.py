@@ -60,6 +60,27 @@ def fd_gradient_error(inp, causal, base, h_rel=1e-5):
     return worst
 
 
+def fd_input_gradient_error(inp, causal, base, h_rel=1e-5):
+    """max over A1, A2, A3 of ||g_fd - g|| / ||g|| with central differences of Loss
+    (every entry of every instance)."""
+    g = oracle.forward_backward(inp, causal, base)
+    worst = 0.0
+    for aname, gname in (("A1", "dA1"), ("A2", "dA2"), ("A3", "dA3")):
+        A = inp[aname]
+        fd = np.zeros_like(A, dtype=float)
+        for idx in np.ndindex(A.shape):
+            a0 = A[idx]
+            step = h_rel * max(1.0, abs(a0))
+            A[idx] = a0 + step
+            lp = oracle.loss_only(inp, causal, base)
+            A[idx] = a0 - step
+            lm = oracle.loss_only(inp, causal, base)
+            A[idx] = a0
+            fd[idx] = (lp - lm) / (2 * step)
+        worst = max(worst, _rel(g[gname], fd))
+    return worst
+
+
 def sdpa_error(inp, causal):
     """Positions all zero: compare O, lse, loss and dW with torch's SDPA + autograd (fp64).
 
@@ -251,6 +272,32 @@ def test_finite_differences(n, d, causal, base):
 def test_finite_differences_batch_and_heads():
     inp = _tiny(4, 4, H=2, B=2, seed=11)
     assert fd_gradient_error(inp, True, 1e4) <= 1e-6
+
+
+@pytest.mark.parametrize("n,d", [(1, 2), (3, 2), (5, 4), (8, 4)])
+@pytest.mark.parametrize("causal", [False, True])
+def test_input_gradient_finite_differences(n, d, causal):
+    """dA1, dA2, dA3 (next row of the scope: input gradients) against central differences."""
+    inp = _tiny(n, d, seed=5 + n)
+    assert fd_input_gradient_error(inp, causal, 1e4) <= 1e-6
+
+
+def test_input_gradient_finite_differences_batch_and_heads():
+    inp = _tiny(3, 4, H=2, B=2, seed=13)
+    assert fd_input_gradient_error(inp, True, 10.0) <= 1e-6
+
+
+def test_planted_input_gradient_untransposed_weight(monkeypatch):
+    """dA1 = dQ WQ (a missing transpose) fails the finite-difference pin."""
+    orig = ra.instance_forward_backward
+
+    def bad(*args, **kw):
+        out = orig(*args, **kw)
+        if "dA1" in out:
+            out["dA1"] = out["dQ"] @ np.asarray(args[4], float)
+        return out
+    monkeypatch.setattr(ra, "instance_forward_backward", bad)
+    assert fd_input_gradient_error(_tiny(3, 4, seed=2), False, 1e4) > 1e-3
 
 
 @pytest.mark.parametrize("causal", [False, True])
