@@ -49,6 +49,7 @@ def parse():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=list(WORKLOADS))
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-input-grads", action="store_true")
     return ap.parse_args()
 
 
@@ -278,6 +279,32 @@ def run_ours(args, rank, world, local_rank):
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "pipelining": "next step's host-to-device copy overlaps this step's compute"}
 
+    # ---- the input-gradient row (rope_attn_loss_bwd_inputs), timed outside the step -----
+    # The metric's step is the forward and the weight-gradient backward; the extra products
+    # dA = dX W^T are measured on their own: the backward with input gradients is run a few
+    # times with per-kernel events and the input-gradient kernel's average launch is kept.
+    input_grads = None
+    if not args.no_input_grads:
+        m.forward()
+        m.backward_inputs(True)
+        torch.cuda.synchronize(dev)
+        ra.profile_read()
+        ra.profile_enable(True)
+        reps = 5
+        for _ in range(reps):
+            m.forward()
+            m.backward_inputs(True)
+        torch.cuda.synchronize(dev)
+        prof_ig = ra.profile_read()
+        ra.profile_enable(False)
+        st = ra.last_error()
+        if st != ra.RA_OK:
+            raise RuntimeError(f"kernel status after the input-gradient run: {ra.status_string(st)}")
+        for kname in ("input_grads_tc", "input_grads_simt"):
+            if kname in prof_ig:
+                ms_ig, n_ig = prof_ig[kname]
+                input_grads = {"kernel": kname, "avg_launch_ms": round(ms_ig / max(1, n_ig), 4)}
+
     if rank != 0:
         return None
 
@@ -301,12 +328,42 @@ def run_ours(args, rank, world, local_rank):
         "kernels": {k: {"ms_per_step": round(v[0] / args.steps, 4),
                         "launches": v[1], "share": round(v[0] / total_kernel_ms, 4)}
                     for k, v in sorted(per_kernel.items(), key=lambda kv: -kv[1][0])},
+        "kernel_rooflines": {k: kernel_roofline(w, k, v[0] / max(1, v[1]), pk)
+                             for k, v in per_kernel.items()
+                             if kernel_roofline(w, k, 1.0, pk) is not None},
         "gpu_launches": int(launches),
         "clocks": clk,
         "e2e": e2e,
         "peaks_source": src,
     }
+    if input_grads is not None:
+        line["input_grads"] = dict(input_grads, **(kernel_roofline(
+            w, input_grads["kernel"], input_grads["avg_launch_ms"], pk) or {}))
     return line
+
+
+def kernel_roofline(w, kname, avg_ms, pk):
+    """Per-kernel roofline of every tensor-core / memory-bound kernel on the path: algorithmic
+    flops (tensor) or bytes (HBM) of one launch over its CUDA-event-timed average duration."""
+    BH, n, d = w.B * w.H, w.n, w.d
+    P = pair_count(n, w.causal)
+    act = BH * n * d                     # elements of one [B][H][n][d] tensor
+    tensor = {"attn_bwd_tc": 10.0 * d * P * BH, "attn_fwd_tc": 4.0 * d * P * BH}
+    # bytes: proj reads A1..A3 and writes Q~, K~, V (bf16); dq_unrotate reads fp32 dQ~ and
+    # writes bf16 dQ; dw_tc reads A1..A3 and dQ, dK, dV (bf16); the input gradients read
+    # dQ, dK, dV and write dA1..dA3 (bf16).  Tables and weights are L2-resident extras.
+    hbm = {"proj_rope_tc": 12.0 * act, "dq_unrotate": 6.0 * act, "dw_tc": 12.0 * act,
+           "input_grads_tc": 12.0 * act}
+    if kname in tensor:
+        ach = tensor[kname] / (avg_ms * 1e-3) / 1e12
+        return {"bound": "tensor", "achieved": round(ach, 3), "peak": pk["bf16_tflops"],
+                "unit": "TFLOP/s", "frac": round(ach / pk["bf16_tflops"], 4),
+                "avg_launch_ms": round(avg_ms, 4)}
+    if kname in hbm:
+        ach = hbm[kname] / (avg_ms * 1e-3) / 1e9
+        return {"bound": "hbm", "achieved": round(ach, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
+                "frac": round(ach / pk["hbm_gbs"], 4), "avg_launch_ms": round(avg_ms, 4)}
+    return None
 
 
 def roofline(w, kname, avg_ms, pk, src):

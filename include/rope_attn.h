@@ -108,6 +108,20 @@ ra_status rope_attn_loss_bwd(const ra_problem* p, const void* O, const float* ls
                              void* ws, size_t ws_bytes, int32_t ws_holds_fwd, void* stream);
 
 /*
+ * rope_attn_loss_bwd followed by the gradients with respect to the three inputs, by the same
+ * chain rule through Q = A1 WQ, K = A2 WK, V = A3 WV (the page's problem stops at the weight
+ * gradients; these let layers be stacked):
+ *   dA1 = rot^-1(dQ~) WQ^T,  dA2 = rot^-1(dK~) WK^T,  dA3 = dV WV^T
+ *   dA1/dA2/dA3 : device [B][H][n][d], element type p->dtype (overwritten); none may be NULL
+ * Other arguments, validation and errors as rope_attn_loss_bwd.  With bf16 I/O the products
+ * use the bf16-rounded dQ, dK, dV (fp32 accumulation).
+ */
+ra_status rope_attn_loss_bwd_inputs(const ra_problem* p, const void* O, const float* lse,
+                                    float* loss, float* dWQ, float* dWK, float* dWV, void* dA1,
+                                    void* dA2, void* dA3, void* ws, size_t ws_bytes,
+                                    int32_t ws_holds_fwd, void* stream);
+
+/*
  * Synchronises `stream`, then reports and clears the device-side status word of the current
  * device: RA_ERR_TIMEOUT if a kernel gave up waiting since the last call, else RA_OK
  * (RA_ERR_CUDA if the synchronisation itself failed).

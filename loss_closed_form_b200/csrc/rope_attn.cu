@@ -40,12 +40,15 @@ enum KernelId : int {
   K_PROJ_TC,
   K_DQ_UNROT,
   K_DW_TC,
+  K_DA_TC,
+  K_DA_SIMT,
   K_COUNT
 };
 const char* const kKernelNames[K_COUNT] = {
     "rope_table", "proj_rope_simt", "attn_fwd_simt", "bwd_pre",
     "attn_bwd_simt", "dw_partial_simt", "dw_reduce", "loss_finalize",
-    "attn_fwd_tc", "attn_bwd_tc", "proj_rope_tc", "dq_unrotate", "dw_tc"};
+    "attn_fwd_tc", "attn_bwd_tc", "proj_rope_tc", "dq_unrotate", "dw_tc",
+    "input_grads_tc", "input_grads_simt"};
 
 struct ProfRecord {
   int id;
@@ -366,10 +369,63 @@ ra_status tc_project(const ra_problem* p, const Layout& L, void* ws, cudaStream_
   pp.tiles_per_cta = (pp.tiles + ctas - 1) / ctas;
   const long long grid = (pp.tiles + pp.tiles_per_cta - 1) / pp.tiles_per_cta;
   pp.limit_ns = wait_limit_ns();
-  auto k = proj_rope_tc_kernel<D>;
+  auto k = proj_rope_tc_kernel<D, false>;
   cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_ALLOC);
   Launch l(K_PROJ_TC, st);
   k<<<(unsigned)grid, C::THREADS, C::SMEM_ALLOC, st>>>(a1, a2, a3, w1, w2, w3, o1, o2, o3, pp);
+  return launch_status();
+}
+
+// Input gradients dA_z = dX_z W_z^T from the bf16 dQ, dK, dV the backward left in the
+// workspace (same persistent tcgen05 kernel as the projections, without rotation).
+template <int D>
+ra_status tc_input_grads(const ra_problem* p, const Layout& L, void* dA1, void* dA2, void* dA3,
+                         void* ws, cudaStream_t st) {
+  using namespace ra::tc;
+  using C = ProjCfg<D>;
+  const int n = p->n, BH = p->B * p->H;
+  CUtensorMap a1, a2, a3, w1, w2, w3, o1, o2, o3;
+  if (!map_bf16_3d(&a1, at<void>(ws, L.dq16), D, n, BH, C::BM) ||
+      !map_bf16_3d(&a2, at<void>(ws, L.dk16), D, n, BH, C::BM) ||
+      !map_bf16_3d(&a3, at<void>(ws, L.dv16), D, n, BH, C::BM) ||
+      !map_bf16_3d(&w1, p->WQ, D, D, p->H, D) || !map_bf16_3d(&w2, p->WK, D, D, p->H, D) ||
+      !map_bf16_3d(&w3, p->WV, D, D, p->H, D) || !map_bf16_3d(&o1, dA1, D, n, BH, C::BM) ||
+      !map_bf16_3d(&o2, dA2, D, n, BH, C::BM) || !map_bf16_3d(&o3, dA3, D, n, BH, C::BM))
+    return RA_ERR_CUDA;
+  ProjParams pp;
+  pp.tab = at<float2>(ws, L.rope);
+  pp.n = n;
+  pp.B = p->B;
+  pp.H = p->H;
+  pp.nrt = (n + C::BM - 1) / C::BM;
+  pp.tiles = (long long)p->B * pp.nrt * 3 * p->H;
+  const long long sms = num_sms();
+  const long long ctas = pp.tiles < sms ? pp.tiles : sms;
+  pp.tiles_per_cta = (pp.tiles + ctas - 1) / ctas;
+  const long long grid = (pp.tiles + pp.tiles_per_cta - 1) / pp.tiles_per_cta;
+  pp.limit_ns = wait_limit_ns();
+  auto k = proj_rope_tc_kernel<D, true>;
+  cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_ALLOC);
+  Launch l(K_DA_TC, st);
+  k<<<(unsigned)grid, C::THREADS, C::SMEM_ALLOC, st>>>(a1, a2, a3, w1, w2, w3, o1, o2, o3, pp);
+  return launch_status();
+}
+
+// fp32 I/O: dA_z = rot^-1(dX~_z) W_z^T on the CUDA cores (dQ~, dK~ are kept rotated there).
+ra_status simt_input_grads(const ra_problem* p, const Layout& L, void* dA1, void* dA2,
+                           void* dA3, void* ws, cudaStream_t st) {
+  const int n = p->n, d = p->d;
+  dim3 grid((n + ra::simt::kDaRows - 1) / ra::simt::kDaRows, p->B * p->H, 3);
+  const size_t smem = (size_t)(d * d + ra::simt::kDaRows * d) * sizeof(float);
+  auto k = ra::simt::input_grad_kernel;
+  if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+      cudaSuccess)
+    return RA_ERR_CUDA;
+  Launch l(K_DA_SIMT, st);
+  k<<<grid, ra::simt::kThreads, smem, st>>>(
+      at<float>(ws, L.dqt), at<float>(ws, L.dkt), at<float>(ws, L.dv), at<float2>(ws, L.rope),
+      (const float*)p->WQ, (const float*)p->WK, (const float*)p->WV, (float*)dA1, (float*)dA2,
+      (float*)dA3, p->H, n, d);
   return launch_status();
 }
 
@@ -650,6 +706,23 @@ ra_status rope_attn_loss_bwd(const ra_problem* p, const void* O, const float* ls
   if (p->dtype == RA_F32)
     return simt_bwd(p, O, lse, loss, dWQ, dWK, dWV, ws, ws_holds_fwd, st);
   return tc_bwd(p, O, lse, loss, dWQ, dWK, dWV, ws, ws_holds_fwd, st);
+}
+
+ra_status rope_attn_loss_bwd_inputs(const ra_problem* p, const void* O, const float* lse,
+                                    float* loss, float* dWQ, float* dWK, float* dWV, void* dA1,
+                                    void* dA2, void* dA3, void* ws, size_t ws_bytes,
+                                    int32_t ws_holds_fwd, void* stream) {
+  if (!p || !dA1 || !dA2 || !dA3) return RA_ERR_INVALID_ARG;
+  if (!is_aligned(dA1, 16) || !is_aligned(dA2, 16) || !is_aligned(dA3, 16))
+    return RA_ERR_ALIGNMENT;
+  ra_status s = rope_attn_loss_bwd(p, O, lse, loss, dWQ, dWK, dWV, ws, ws_bytes, ws_holds_fwd,
+                                   stream);
+  if (s != RA_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const Layout L = make_layout(p);
+  if (p->dtype == RA_F32) return simt_input_grads(p, L, dA1, dA2, dA3, ws, st);
+  return p->d == 128 ? tc_input_grads<128>(p, L, dA1, dA2, dA3, ws, st)
+                     : tc_input_grads<64>(p, L, dA1, dA2, dA3, ws, st);
 }
 
 ra_status rope_attn_step_noalloc(const ra_problem* p, void* O, float* lse, float* loss,

@@ -459,5 +459,59 @@ __global__ void loss_finalize_kernel(const double* __restrict__ part, int count,
   if (threadIdx.x == 0) *loss = (float)red[0];
 }
 
+// ---------------------------------------------------------------------------------------
+// Input gradients (fp32 I/O): dA_z[b, h, i, :] = rot^-1(dX~_z[b, h, i, :]) W_z[h]^T, with
+// z = 0 (dQ~, rotated), 1 (dK~, rotated), 2 (dV).  grid (row blocks, B * H, 3); W_z[h] is
+// transposed into shared memory so the 16 threads of a row read consecutive words.
+// ---------------------------------------------------------------------------------------
+constexpr int kDaRows = 16;
+
+__global__ void __launch_bounds__(kThreads)
+input_grad_kernel(const float* __restrict__ dQt, const float* __restrict__ dKt,
+                  const float* __restrict__ dV, const float2* __restrict__ tab,
+                  const float* __restrict__ WQ, const float* __restrict__ WK,
+                  const float* __restrict__ WV, float* __restrict__ dA1, float* __restrict__ dA2,
+                  float* __restrict__ dA3, int H, int n, int d) {
+  extern __shared__ float smem[];
+  float* Wt = smem;          // [d][d]: Wt[o][a] = W[a][o]
+  float* Xs = smem + d * d;  // [kDaRows][d]: un-rotated rows of dX
+  const int z = blockIdx.z, bh = blockIdx.y, h = bh % H;
+  const int r0 = blockIdx.x * kDaRows;
+  const float* X = z == 0 ? dQt : z == 1 ? dKt : dV;
+  const float* W = (z == 0 ? WQ : z == 1 ? WK : WV) + (size_t)h * d * d;
+  float* dA = z == 0 ? dA1 : z == 1 ? dA2 : dA3;
+  for (int e = threadIdx.x; e < d * d; e += blockDim.x) {
+    const int a = e / d, o = e - a * d;
+    Wt[o * d + a] = W[e];
+  }
+  const int half = d / 2;
+  for (int e = threadIdx.x; e < kDaRows * half; e += blockDim.x) {
+    const int rr = e / half, k = e - rr * half, i = r0 + rr;
+    float x0 = 0.f, x1 = 0.f;
+    if (i < n) {
+      const size_t off = ((size_t)bh * n + i) * d + 2 * k;
+      const float y0 = X[off], y1 = X[off + 1];
+      if (z < 2) {
+        const float2 cs = tab[(size_t)i * half + k];  // rotation by -phi
+        x0 = y0 * cs.x + y1 * cs.y;
+        x1 = -y0 * cs.y + y1 * cs.x;
+      } else {
+        x0 = y0;
+        x1 = y1;
+      }
+    }
+    Xs[rr * d + 2 * k] = x0;
+    Xs[rr * d + 2 * k + 1] = x1;
+  }
+  __syncthreads();
+  const int rr = threadIdx.x / 16, a0 = threadIdx.x % 16, i = r0 + rr;
+  if (i >= n) return;
+  for (int a = a0; a < d; a += 16) {
+    float acc = 0.f;
+    for (int o = 0; o < d; ++o) acc = fmaf(Xs[rr * d + o], Wt[o * d + a], acc);
+    dA[((size_t)bh * n + i) * d + a] = acc;
+  }
+}
+
 }  // namespace simt
 }  // namespace ra

@@ -20,7 +20,8 @@ namespace tc {
 // ---------------------------------------------------------------------------------------
 // Persistent kernel over 128-row tiles ordered (row tile, z, head) with the head fastest, so
 // a CTA keeps one row tile's RoPE angles (cos, sin) in registers while it runs through the
-// heads.  Per tile: TMA loads A_z[b, h] rows and W_z[h]; one tcgen05 product into a
+// heads.  With IG (input gradients) the same kernel computes dA_z = dX_z W_z^T from the
+// un-rotated dQ, dK, dV: W is then read as a K-major B operand and nothing is rotated.  Per tile: TMA loads A_z[b, h] rows and W_z[h]; one tcgen05 product into a
 // double-buffered TMEM accumulator; the epilogue warps rotate, round to bf16 and write a
 // 128-byte-swizzled staging tile that a TMA store sends to global memory (the staging is
 // double-buffered, so the store of one tile overlaps the next tile's epilogue).
@@ -59,7 +60,7 @@ struct ProjParams {
   unsigned long long limit_ns;
 };
 
-template <int D>
+template <int D, bool IG>
 __global__ void __launch_bounds__(ProjCfg<D>::THREADS, 1)
 proj_rope_tc_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_constant__ CUtensorMap tm_a2,
                     const __grid_constant__ CUtensorMap tm_a3, const __grid_constant__ CUtensorMap tm_w1,
@@ -149,7 +150,9 @@ proj_rope_tc_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_cons
   } else if (warp == C::W_MMA) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16_f32(128, D, false, true);
+      // X = A W: W[in][out] is the B operand (K = in, N = out contiguous: MN-major).
+      // dA = dX W^T: B[k = out][n = in] = W[in][out] (K contiguous: K-major).
+      constexpr uint32_t idesc = idesc_bf16_f32(128, D, false, !IG);
       bool ok = true;
       for (int t = 0; ok && t < NT; ++t) {
         const int s = t % C::NS, ab = t & 1;
@@ -159,9 +162,12 @@ proj_rope_tc_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_cons
         const uint32_t a = sbase + C::A_OFF + s * C::ATILE;
         const uint32_t w = sbase + C::W_OFF + s * C::WTILE;
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk)
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint64_t bdesc = IG ? sw128_desc(w + (kk >> 2) * C::WBLK + (kk & 3) * 32, 16, 1024)
+                                    : sw128_desc(w + kk * 2048, C::WBLK, 1024);
           mma_ss(tmem + ab * D, sw128_desc(a + (kk >> 2) * C::ABLK + (kk & 3) * 32, 16, 1024),
-                 sw128_desc(w + kk * 2048, C::WBLK, 1024), idesc, kk > 0);
+                 bdesc, idesc, kk > 0);
+        }
         mma_commit(b_accfull(ab));
         mma_commit(b_ldempty(s));
       }
@@ -200,7 +206,7 @@ proj_rope_tc_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_cons
       int b, rt, z, h;
       decode(t, b, rt, z, h);
       const int row = rt * C::BM + rl;
-      if (z < 2 && rt != key) {
+      if (!IG && z < 2 && rt != key) {
         key = rt;
         const float4* tr = reinterpret_cast<const float4*>(p.tab + (size_t)(row < p.n ? row : 0) * (D / 2) + c0 / 2);
 #pragma unroll
@@ -229,7 +235,7 @@ proj_rope_tc_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_cons
 #pragma unroll
         for (int k2 = 0; k2 < 4; ++k2) {
           float x0 = __uint_as_float(r[8 * c + 2 * k2]), x1 = __uint_as_float(r[8 * c + 2 * k2 + 1]);
-          if (z < 2) {
+          if (!IG && z < 2) {
             const float2 a = cs[4 * c + k2];
             const float y0 = x0 * a.x - x1 * a.y, y1 = x0 * a.y + x1 * a.x;
             x0 = y0;

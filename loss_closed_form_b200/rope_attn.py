@@ -21,7 +21,7 @@ RA_F32, RA_BF16 = 0, 1
 EXPORTED = ("rope_attn_workspace_bytes", "rope_attn_fwd", "rope_attn_loss_bwd",
             "rope_attn_last_error", "rope_attn_status_string", "rope_attn_launch_count",
             "rope_attn_profile_enable", "rope_attn_profile_read", "rope_attn_kernel_name",
-            "rope_attn_step_noalloc")
+            "rope_attn_step_noalloc", "rope_attn_loss_bwd_inputs")
 
 # Capacity of the static scratch behind rope_attn_step_noalloc (RA_NOALLOC_SCRATCH_BYTES).
 NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
@@ -79,6 +79,9 @@ def load() -> ctypes.CDLL:
     lib.rope_attn_kernel_name.restype = ctypes.c_char_p
     lib.rope_attn_step_noalloc.argtypes = [P, vp, vp, vp, vp, vp, vp, vp]
     lib.rope_attn_step_noalloc.restype = ctypes.c_int
+    lib.rope_attn_loss_bwd_inputs.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz,
+                                              i32, vp]
+    lib.rope_attn_loss_bwd_inputs.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -148,6 +151,17 @@ def loss_bwd(prob: Problem, O, lse, loss, dWQ, dWK, dWV, ws, ws_holds_fwd=False,
                                    _stream(stream))
     if st != RA_OK:
         raise RopeAttnError(st, "rope_attn_loss_bwd")
+
+
+def loss_bwd_inputs(prob: Problem, O, lse, loss, dWQ, dWK, dWV, dA1, dA2, dA3, ws,
+                    ws_holds_fwd=False, stream=None) -> None:
+    """rope_attn_loss_bwd_inputs: as loss_bwd, plus dA1, dA2, dA3 ([B][H][n][d], I/O dtype)."""
+    st = load().rope_attn_loss_bwd_inputs(
+        ctypes.byref(prob), _ptr(O), _ptr(lse), _ptr(loss), _ptr(dWQ), _ptr(dWK), _ptr(dWV),
+        _ptr(dA1), _ptr(dA2), _ptr(dA3), _ptr(ws), ws.numel() * ws.element_size(),
+        int(bool(ws_holds_fwd)), _stream(stream))
+    if st != RA_OK:
+        raise RopeAttnError(st, "rope_attn_loss_bwd_inputs")
 
 
 def step_noalloc(prob: Problem, O, lse, loss, dWQ, dWK, dWV, stream=None) -> None:
@@ -230,6 +244,17 @@ class RopeAttention:
         loss_bwd(self.prob, self.O, self.lse, self.loss, self.dWQ, self.dWK, self.dWV, self.ws,
                  ws_holds_fwd, stream)
         return self.loss, self.dWQ, self.dWK, self.dWV
+
+    def backward_inputs(self, ws_holds_fwd=True, stream=None):
+        """Backward with the input gradients: returns (loss, dWQ, dWK, dWV, dA1, dA2, dA3)."""
+        import torch
+        if not hasattr(self, "dA1"):
+            self.dA1 = torch.empty_like(self.O)
+            self.dA2 = torch.empty_like(self.O)
+            self.dA3 = torch.empty_like(self.O)
+        loss_bwd_inputs(self.prob, self.O, self.lse, self.loss, self.dWQ, self.dWK, self.dWV,
+                        self.dA1, self.dA2, self.dA3, self.ws, ws_holds_fwd, stream)
+        return self.loss, self.dWQ, self.dWK, self.dWV, self.dA1, self.dA2, self.dA3
 
     def step(self, stream=None):
         self.forward(stream)
