@@ -265,6 +265,21 @@ bool map_bf16_3d(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows,
          CUDA_SUCCESS;
 }
 
+// 2-D map over fp32 rows [rows][cols] with boxes of 32 columns (128 bytes) x box_rows,
+// 128-byte swizzle (the RoPE table rows of a tile, read back with swizzled shared loads).
+bool map_f32_rows_sw128(CUtensorMap* m, void* base, uint64_t cols, uint64_t rows,
+                        uint32_t box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 4};
+  cuuint32_t box[2] = {32, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, base, dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // 3-D map over fp32 rows [outer][rows][cols] with a box of cols x box_rows, no swizzle
 // (the target of bulk reductions).
 bool map_f32_3d(CUtensorMap* m, void* base, uint64_t cols, uint64_t rows, uint64_t outer,
@@ -528,19 +543,19 @@ ra_status tc_bwd_launch(const ra_problem* p, const Layout& L, const float* lse, 
   using namespace ra::tc;
   using C = BwdCfg<D>;
   const int n = p->n, BH = p->B * p->H;
-  CUtensorMap mq, mk, mv, ml, mdq;
+  CUtensorMap mq, mk, mv, ml, mdq, mtab, mdk, mdv;
   if (!map_bf16_3d(&mq, at<void>(ws, L.qt), D, n, BH, C::BQ) ||
       !map_bf16_3d(&mk, at<void>(ws, L.kt), D, n, BH, C::BK) ||
       !map_bf16_3d(&mv, at<void>(ws, L.v), D, n, BH, C::BK) ||
       !map_bf16_3d(&ml, at<void>(ws, L.ell), D, n, BH, C::BQ) ||
-      !map_f32_3d(&mdq, at<void>(ws, L.dqt), D, n, BH, C::BQ))
+      !map_f32_3d(&mdq, at<void>(ws, L.dqt), D, n, BH, C::BQ) ||
+      !map_f32_rows_sw128(&mtab, at<void>(ws, L.rope), D, n, C::BK) ||
+      !map_bf16_3d(&mdk, at<void>(ws, L.dk16), D, n, BH, C::BK) ||
+      !map_bf16_3d(&mdv, at<void>(ws, L.dv16), D, n, BH, C::BK))
     return RA_ERR_CUDA;
   BwdParams bp;
   bp.lse = lse;
   bp.delta = at<float>(ws, L.delta);
-  bp.tab = at<float2>(ws, L.rope);
-  bp.dK = at<__nv_bfloat16>(ws, L.dk16);
-  bp.dV = at<__nv_bfloat16>(ws, L.dv16);
   bp.n = n;
   bp.BH = BH;
   bp.nk = (n + C::BK - 1) / C::BK;
@@ -552,7 +567,7 @@ ra_status tc_bwd_launch(const ra_problem* p, const Layout& L, const float* lse, 
   cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_ALLOC);
   dim3 grid(bp.nk, BH);
   Launch l(K_BWD_TC, st);
-  k<<<grid, C::THREADS, C::SMEM_ALLOC, st>>>(mq, mk, mv, ml, mdq, bp);
+  k<<<grid, C::THREADS, C::SMEM_ALLOC, st>>>(mq, mk, mv, ml, mdq, mtab, mdk, mdv, bp);
   return RA_OK;
 }
 

@@ -52,11 +52,16 @@ struct BwdCfg {
   static constexpr int BAR_OFF = LD_OFF + NSQ * BQ * 8;
   // kv_full, q_full[NSQ], q_empty[NSQ], s_full, s_free, pg_full, pg_free, dq_full, dq_free,
   // acc_done, drain, dqs_full, dqs_free
-  static constexpr int NBAR = 1 + 2 * NSQ + 10;
+  static constexpr int NBAR = 1 + 2 * NSQ + 12;   // ... + tab_full, ep_full
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
   static constexpr int SMEM_USED = MISC_OFF + 64;
   static constexpr int SMEM_ALLOC =
       (SMEM_USED + 1024 > 120 * 1024) ? SMEM_USED + 1024 : 120 * 1024;
+  // epilogue: the (cos, sin) rows of the key tile as D / 32 boxes of [128 rows][128 bytes]
+  // (128-byte swizzle) over K~ / V, and dK / dV staged over the query-tile stages
+  static constexpr int TBLK = BK * 128;
+  static constexpr int TABT = BK * D * 4;
+  static_assert(TABT <= 2 * KTILE && 2 * KTILE <= 2 * NSQ * QTILE, "epilogue staging");
   static constexpr int THREADS = 448;
   static constexpr int W_DRAIN = 8, W_PROD = 12, W_MMA = 13;
   // TMEM columns
@@ -69,9 +74,6 @@ struct BwdCfg {
 struct BwdParams {
   const float* lse;     // [BH][n]
   const float* delta;   // [BH][n]
-  const float2* tab;    // [n][d/2] (cos, sin) of the RoPE angles
-  __nv_bfloat16* dK;    // [BH][n][d] rot^-1(dK~), bf16
-  __nv_bfloat16* dV;    // [BH][n][d] bf16
   int n, BH, nk, causal;
   float scale;         // 1 / sqrt(d)
   float scale_log2;    // log2(e) / sqrt(d)
@@ -82,7 +84,9 @@ template <int D>
 __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
 attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_l,
-                   const __grid_constant__ CUtensorMap tm_dq, const BwdParams p) {
+                   const __grid_constant__ CUtensorMap tm_dq, const __grid_constant__ CUtensorMap tm_tab,
+                   const __grid_constant__ CUtensorMap tm_dk, const __grid_constant__ CUtensorMap tm_dv,
+                   const BwdParams p) {
   using C = BwdCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -105,6 +109,8 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
   const uint32_t b_drain = smem_u32(&bars[8 + 2 * C::NSQ]);
   const uint32_t b_dqsfull = smem_u32(&bars[9 + 2 * C::NSQ]);
   const uint32_t b_dqsfree = smem_u32(&bars[10 + 2 * C::NSQ]);
+  const uint32_t b_tab = smem_u32(&bars[11 + 2 * C::NSQ]);  // RoPE rows of the key tile landed
+  const uint32_t b_ep = smem_u32(&bars[12 + 2 * C::NSQ]);   // dK / dV staging written
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   // head-major order: the key tiles of one (b, h) run side by side and share its Q~, l and
@@ -133,6 +139,8 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     mbar_init(b_drain, 1);
     mbar_init(b_dqsfull, 128);
     mbar_init(b_dqsfree, 1);
+    mbar_init(b_tab, 1);
+    mbar_init(b_ep, 256);
     abort_set(abort_flag, 0);
     fence_barrier_init();
   }
@@ -316,37 +324,59 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       mbar_arrive(b_pgfull);
     }
     // ---- dK = rot^-1(scale * sum gamma^T Q~) (warps 0-3), dV = sum P^T l (warps 4-7):
-    //      one key row per thread
+    //      one key row per thread.  Once every product has completed, K~, V and the query
+    //      stages are free: the RoPE (cos, sin) rows of this key tile come in by TMA over
+    //      K~ / V, and dK, dV are staged (128-byte swizzle) over the query stages and leave by
+    //      TMA stores (per-thread rows of 16-byte accesses would be uncoalesced).
     if (ok) ok = mbar_wait_warp(b_acc, 0, abort_flag, lim);
+    const uint32_t tab_s = sbase + C::K_OFF;
+    const uint32_t stg = sbase + C::Q_OFF + half * C::KTILE;
+    if (ok && tid == 0) {
+      mbar_expect_tx(b_tab, C::TABT);
+      for (int b = 0; b < D / 32; ++b)
+        tma_load_2d(tab_s + b * C::TBLK, &tm_tab, b_tab, 32 * b, kt * C::BK);
+    }
+    if (ok && half == 0) ok = mbar_wait_warp(b_tab, 0, abort_flag, lim);
     if (ok) {
       tc_fence_after();
-      const size_t ro = ((size_t)bh * n + key) * D;
-      const float2* tr = p.tab + (size_t)(key < n ? key : 0) * (D / 2);
-      __nv_bfloat16* dst = (half == 0 ? p.dK : p.dV) + ro;
       const uint32_t src = tmem + lane_base + (half == 0 ? C::T_DK : C::T_DV);
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t r[32];
         tmem_ld32(src + 32 * c, r);
         tmem_wait_ld();
-        if (key < n) {
-          uint32_t w[16];
+        uint32_t w[16];
 #pragma unroll
-          for (int k = 0; k < 16; ++k) {
-            const float x0 = __uint_as_float(r[2 * k]), x1 = __uint_as_float(r[2 * k + 1]);
-            if (half == 0) {
-              const float y0 = x0 * p.scale, y1 = x1 * p.scale;
-              const float2 cs = tr[16 * c + k];  // rotation by -phi
-              w[k] = pack_bf16x2(y0 * cs.x + y1 * cs.y, -y0 * cs.y + y1 * cs.x);
-            } else {
-              w[k] = pack_bf16x2(x0, x1);
-            }
+        for (int k = 0; k < 16; k += 2) {
+          const float x0 = __uint_as_float(r[2 * k]), x1 = __uint_as_float(r[2 * k + 1]);
+          const float x2 = __uint_as_float(r[2 * k + 2]), x3 = __uint_as_float(r[2 * k + 3]);
+          if (half == 0) {
+            // pairs 16 c + k, 16 c + k + 1: (cos, sin, cos, sin), rotation by -phi
+            const float4 cs = ld_shared_v4f(tab_s + c * C::TBLK + sw128_offset(row, k >> 1));
+            const float y0 = x0 * p.scale, y1 = x1 * p.scale, y2 = x2 * p.scale, y3 = x3 * p.scale;
+            w[k] = pack_bf16x2(y0 * cs.x + y1 * cs.y, -y0 * cs.y + y1 * cs.x);
+            w[k + 1] = pack_bf16x2(y2 * cs.z + y3 * cs.w, -y2 * cs.w + y3 * cs.z);
+          } else {
+            w[k] = pack_bf16x2(x0, x1);
+            w[k + 1] = pack_bf16x2(x2, x3);
           }
-          uint4* o = reinterpret_cast<uint4*>(dst + 32 * c);
-#pragma unroll
-          for (int v = 0; v < 4; ++v) o[v] = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
         }
+        // output columns 32 c .. 32 c + 31: 64-column box c / 2, 16-byte chunks 4 (c % 2) ..
+#pragma unroll
+        for (int v = 0; v < 4; ++v)
+          st_shared_v4(stg + (c >> 1) * C::KBLK + sw128_offset(row, 4 * (c & 1) + v), w[4 * v],
+                       w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
       }
+    }
+    fence_proxy_async_smem();
+    mbar_arrive(b_ep);
+    if (tid == 0 && ok && mbar_wait(b_ep, 0, abort_flag, lim)) {
+      for (int b = 0; b < D / 64; ++b) {
+        tma_store_3d(&tm_dk, sbase + C::Q_OFF + b * C::KBLK, 64 * b, kt * C::BK, bh);
+        tma_store_3d(&tm_dv, sbase + C::Q_OFF + C::KTILE + b * C::KBLK, 64 * b, kt * C::BK, bh);
+      }
+      bulk_commit();
+      bulk_wait0();  // the stores have landed before the CTA leaves
     }
   } else {
     // ------------------------------------------------------------------ dQ~ drain (warps 8-11)
