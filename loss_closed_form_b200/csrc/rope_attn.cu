@@ -494,10 +494,13 @@ ra_status tc_fwd_launch(const ra_problem* p, const Layout& L, void* O, float* ls
   using namespace ra::tc;
   using C = FwdCfg<D>;
   const int n = p->n, BH = p->B * p->H;
-  CUtensorMap mq, mk, mv;
+  CUtensorMap mq, mk, mv, me, mo, mell;
+  // without a target the E map is a placeholder over l (never read: the kernel checks p.E)
   if (!map_bf16_3d(&mq, at<void>(ws, L.qt), D, n, BH, 128) ||
       !map_bf16_3d(&mk, at<void>(ws, L.kt), D, n, BH, 128) ||
-      !map_bf16_3d(&mv, at<void>(ws, L.v), D, n, BH, 128))
+      !map_bf16_3d(&mv, at<void>(ws, L.v), D, n, BH, 128) ||
+      !map_bf16_3d(&me, p->E ? const_cast<void*>(p->E) : at<void>(ws, L.ell), D, n, BH, 128) ||
+      !map_bf16_3d(&mo, O, D, n, BH, 128) || !map_bf16_3d(&mell, at<void>(ws, L.ell), D, n, BH, 128))
     return RA_ERR_CUDA;
   FwdParams fp;
   fp.E = (const __nv_bfloat16*)p->E;
@@ -517,7 +520,7 @@ ra_status tc_fwd_launch(const ra_problem* p, const Layout& L, void* O, float* ls
   cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_ALLOC);
   dim3 grid(fp.npair, BH);
   Launch l(K_FWD_TC, st);
-  k<<<grid, C::THREADS, C::SMEM_ALLOC, st>>>(mq, mk, mv, fp);
+  k<<<grid, C::THREADS, C::SMEM_ALLOC, st>>>(mq, mk, mv, me, mo, mell, fp);
   return RA_OK;
 }
 

@@ -43,8 +43,8 @@ struct FwdCfg {
   static constexpr int V_OFF = K_OFF + NS * TILE;
   static constexpr int BAR_OFF = V_OFF + NS * TILE;
   // barriers: q_full, k_full[NS], k_empty[NS], v_full[NS], v_empty[NS], s_full[2],
-  //           p_full[2], pv_done[2], drain
-  static constexpr int NBAR = 1 + 4 * NS + 6 + 1;
+  //           p_full[2], pv_done[2], drain, e_full[2]
+  static constexpr int NBAR = 1 + 4 * NS + 6 + 1 + 2;
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;  // tmem slot, abort flag
   static constexpr int SMEM_USED = MISC_OFF + 16;
   // at least half of the SM's shared memory: one CTA per SM, so the 512-column TMEM
@@ -78,7 +78,10 @@ template <int D>
 __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
 attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                    const __grid_constant__ CUtensorMap tm_k,
-                   const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
+                   const __grid_constant__ CUtensorMap tm_v,
+                   const __grid_constant__ CUtensorMap tm_e,
+                   const __grid_constant__ CUtensorMap tm_o,
+                   const __grid_constant__ CUtensorMap tm_ell, const FwdParams p) {
   using C = FwdCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -97,6 +100,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
   auto b_pfull = [&](int t) { return smem_u32(&bars[3 + 4 * C::NS + t]); };
   auto b_pvdone = [&](int t) { return smem_u32(&bars[5 + 4 * C::NS + t]); };
   const uint32_t b_drain = smem_u32(&bars[7 + 4 * C::NS]);
+  auto b_efull = [&](int t) { return smem_u32(&bars[8 + 4 * C::NS + t]); };  // E tile landed
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   // head-major order: the query tiles of one (b, h) run side by side and share its K~, V in
@@ -125,6 +129,8 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
       mbar_init(b_pvdone(t), 1);
     }
     mbar_init(b_drain, 1);
+    mbar_init(b_efull(0), 1);
+    mbar_init(b_efull(1), 1);
     abort_set(abort_flag, 0);
     fence_barrier_init();
   }
@@ -333,55 +339,91 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
       tc_fence_before();
       mbar_arrive(b_pfull(t));
     }
-    // ---- epilogue: one full row of O per thread
+    // ---- epilogue: one full row of O per thread.  The tile's query buffer is free (every
+    //      S_t has completed): E_t comes in there by TMA, each thread overwrites its own row
+    //      of E with its row of O (128-byte swizzle), one TMA store sends O out, then l = O - E
+    //      follows the same way.  Rows are private to their thread, so only the hand-overs to
+    //      the storing thread need a barrier (named barrier 1 + t over the warpgroup's 128
+    //      threads, reached the same number of times by every thread).
     float sq = 0.f, dl = 0.f;
     if (ok) ok = mbar_wait_warp(b_pvdone(t), (Tt - 1) & 1, abort_flag, lim);
     const bool vrow = row < n;
+    const uint32_t stg = sbase + C::Q_OFF + t * C::TILE;
+    const bool has_e = p.E != nullptr;
+    if (ok && r == 0 && has_e) {
+      mbar_expect_tx(b_efull(t), C::TILE);
+      for (int b = 0; b < C::KB; ++b)
+        tma_load_3d(stg + b * C::BLK, &tm_e, b_efull(t), 64 * b, qt * C::BM, bh);
+    }
+    if (ok && has_e) ok = mbar_wait_warp(b_efull(t), 0, abort_flag, lim);
+    uint32_t lw[D / 2];  // l = O - E of this row, bf16 pairs
     if (ok) {
       tc_fence_after();
       const float inv_l = 1.f / l;
-      const size_t ro = ((size_t)bh * n + row) * D;
-#pragma unroll 1
+#pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t rr[32];
         tmem_ld32(o_col + 32 * c, rr);
         tmem_wait_ld();
-        if (vrow) {
-          float o[32];
 #pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = __uint_as_float(rr[i]) * inv_l;
-          uint4* Og = reinterpret_cast<uint4*>(p.O + ro + 32 * c);
+        for (int v = 0; v < 4; ++v) {
+          const uint32_t a = stg + (c >> 1) * C::BLK + sw128_offset(r, 4 * (c & 1) + v);
+          float o[8];
 #pragma unroll
-          for (int v = 0; v < 4; ++v)
-            Og[v] = make_uint4(pack_bf16x2(o[8 * v], o[8 * v + 1]), pack_bf16x2(o[8 * v + 2], o[8 * v + 3]),
-                               pack_bf16x2(o[8 * v + 4], o[8 * v + 5]), pack_bf16x2(o[8 * v + 6], o[8 * v + 7]));
-          if (p.E) {
-            const uint4* Eg = reinterpret_cast<const uint4*>(p.E + ro + 32 * c);
-            uint4* Lg = reinterpret_cast<uint4*>(p.ell + ro + 32 * c);
+          for (int i = 0; i < 8; ++i) o[i] = __uint_as_float(rr[8 * v + i]) * inv_l;
+          if (has_e) {
+            const float4 ev = ld_shared_v4f(a);
+            const uint32_t ew[4] = {__float_as_uint(ev.x), __float_as_uint(ev.y),
+                                    __float_as_uint(ev.z), __float_as_uint(ev.w)};
 #pragma unroll
-            for (int v = 0; v < 4; ++v) {
-              const uint4 ev = Eg[v];
-              const uint32_t ew[4] = {ev.x, ev.y, ev.z, ev.w};
-              uint32_t lw[4];
-#pragma unroll
-              for (int q = 0; q < 4; ++q) {
-                const __nv_bfloat162 e2 = *reinterpret_cast<const __nv_bfloat162*>(&ew[q]);
-                const float e0 = o[8 * v + 2 * q] - __low2float(e2);
-                const float e1 = o[8 * v + 2 * q + 1] - __high2float(e2);
-                dl = fmaf(e0, o[8 * v + 2 * q], fmaf(e1, o[8 * v + 2 * q + 1], dl));
+            for (int q = 0; q < 4; ++q) {
+              const __nv_bfloat162 e2 = *reinterpret_cast<const __nv_bfloat162*>(&ew[q]);
+              const float e0 = o[2 * q] - __low2float(e2);
+              const float e1 = o[2 * q + 1] - __high2float(e2);
+              if (vrow) {
+                dl = fmaf(e0, o[2 * q], fmaf(e1, o[2 * q + 1], dl));
                 sq = fmaf(e0, e0, fmaf(e1, e1, sq));
-                lw[q] = pack_bf16x2(e0, e1);
               }
-              Lg[v] = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+              lw[16 * c + 4 * v + q] = pack_bf16x2(e0, e1);
             }
           }
+          st_shared_v4(a, pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]),
+                       pack_bf16x2(o[4], o[5]), pack_bf16x2(o[6], o[7]));
         }
       }
       if (vrow) {
         p.lse[(size_t)bh * n + row] = (m + log2f(l)) * kLn2;
-        if (p.E) p.delta[(size_t)bh * n + row] = dl;
+        if (has_e) p.delta[(size_t)bh * n + row] = dl;
       }
     }
+    fence_proxy_async_smem();
+    named_bar_sync(1 + t, 128);
+    if (ok && r == 0) {
+      for (int b = 0; b < C::KB; ++b)
+        tma_store_3d(&tm_o, stg + b * C::BLK, 64 * b, qt * C::BM, bh);
+      bulk_commit();
+      bulk_wait_read0();
+    }
+    if (has_e) {
+      named_bar_sync(1 + t, 128);  // the O store has read the staging
+      if (ok) {
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c)
+#pragma unroll
+          for (int v = 0; v < 4; ++v)
+            st_shared_v4(stg + (c >> 1) * C::BLK + sw128_offset(r, 4 * (c & 1) + v),
+                         lw[16 * c + 4 * v], lw[16 * c + 4 * v + 1], lw[16 * c + 4 * v + 2],
+                         lw[16 * c + 4 * v + 3]);
+      }
+      fence_proxy_async_smem();
+      named_bar_sync(1 + t, 128);
+      if (ok && r == 0) {
+        for (int b = 0; b < C::KB; ++b)
+          tma_store_3d(&tm_ell, stg + b * C::BLK, 64 * b, qt * C::BM, bh);
+        bulk_commit();
+      }
+    }
+    if (ok && r == 0) bulk_wait0();  // the stores have landed before the CTA leaves
     // per-warp partial of 1/2 sum l^2 (fixed order: deterministic)
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
