@@ -20,5 +20,8 @@ from .rope_attention import (  # noqa: F401
     loss_only,
     scores_rows,
     forward_rows,
+    rotation_matrix,
+    combined_weight_literal,
+    combined_weight_forward_backward,
     ORACLE_PARITY_PINNED,
 )

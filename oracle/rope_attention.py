@@ -247,3 +247,71 @@ def forward_rows(inp: Dict[str, np.ndarray], b: int, h: int, rows, causal: bool,
     gamma = gamma_closed_form(s, beta)
     dQt = (gamma @ Kt) / math.sqrt(d)
     return {"O": O, "lse": lse, "dQt": dQt}
+
+
+# ---------------------------------------------------------------------------------------
+# One combined weight X (the page's own parameterisation)
+# ---------------------------------------------------------------------------------------
+# The page's problem takes the gradient with respect to one vectorised weight x and writes
+# it as dLoss/dx = A~^T vec(gamma(x)) (Probleemdefinitie, Methodologie 1).  Reading: x is
+# vec(X) for the score z_ij = a1_i^T R_{j-i} X a2_j / sqrt(d), where R_{j-i} rotates each
+# pair (2k, 2k+1) by (pos_j - pos_i) * theta_k; a row of A~ is then the derivative of z_ij
+# with respect to X, R_{j-i}^T a1_i a2_j^T / sqrt(d).  Since R_{j-i} = R_i^T R_j, the same
+# scores come from Q~ = rot(A1) and K~ = rot(A2 X^T): the general problem with WQ = I and
+# WK = X^T, whose dWK is dX^T.
+
+
+def rotation_matrix(angles: np.ndarray) -> np.ndarray:
+    """d x d block-diagonal counter-clockwise rotation by ``angles`` (one per pair)."""
+    d = 2 * len(angles)
+    R = np.zeros((d, d), F64)
+    c, s = np.cos(angles), np.sin(angles)
+    for k in range(len(angles)):
+        R[2 * k, 2 * k], R[2 * k, 2 * k + 1] = c[k], -s[k]
+        R[2 * k + 1, 2 * k], R[2 * k + 1, 2 * k + 1] = s[k], c[k]
+    return R
+
+
+def combined_weight_literal(A1, A2, A3, E, X, WV, pos, causal: bool, base: float):
+    """Loss, dLoss/dX and dLoss/dWV of one instance with the page's closed form, literally:
+    the scores from a1_i^T R_{j-i} X a2_j / sqrt(d), s, l, beta, gamma as in
+    ``instance_forward_backward``, then vec(dX) = A~^T vec(gamma) with A~ built row by row
+    (n^2 x d^2: tiny n only)."""
+    A1, A2, A3, E, X, WV = (np.asarray(a, F64) for a in (A1, A2, A3, E, X, WV))
+    n, d = A1.shape
+    c = 1.0 / math.sqrt(d)
+    theta = rope_theta(d, base)
+    p = np.asarray(pos, F64)
+    Rel = [[rotation_matrix((p[j] - p[i]) * theta) for j in range(n)] for i in range(n)]
+    Z = np.empty((n, n), F64)
+    for i in range(n):
+        for j in range(n):
+            Z[i, j] = c * A1[i] @ Rel[i][j] @ X @ A2[j]
+    if causal:
+        Z = np.where(np.arange(n)[None, :] > np.arange(n)[:, None], -np.inf, Z)
+    s, _ = softmax_rows(Z)
+    V = A3 @ WV
+    O = s @ V
+    ell = O - E
+    loss = 0.5 * float(np.sum(ell * ell))
+    beta = ell @ V.T
+    gamma = gamma_closed_form(s, beta)
+    A_tilde = np.empty((n * n, d * d), F64)
+    for i in range(n):
+        for j in range(n):
+            A_tilde[i * n + j] = c * np.outer(Rel[i][j].T @ A1[i], A2[j]).reshape(-1)
+    dX = (A_tilde.T @ gamma.reshape(-1)).reshape(d, d)
+    dWV = A3.T @ (s.T @ ell)
+    return {"loss": loss, "dX": dX, "dWV": dWV, "O": O}
+
+
+def combined_weight_forward_backward(inp: Dict[str, np.ndarray], causal: bool, base: float):
+    """All instances with one combined weight X [H][d][d] per head (``inp["X"]``) through
+    the general problem with WQ = I and WK = X^T: loss, O, dX = dWK^T, dWV."""
+    H, d = inp["X"].shape[0], inp["X"].shape[1]
+    gen = dict(inp)
+    gen["WQ"] = np.broadcast_to(np.eye(d), (H, d, d)).copy()
+    gen["WK"] = np.ascontiguousarray(np.transpose(np.asarray(inp["X"], F64), (0, 2, 1)))
+    r = forward_backward(gen, causal, base)
+    return {"loss": r["loss"], "O": r["O"], "lse": r["lse"],
+            "dX": np.transpose(r["dWK"], (0, 2, 1)), "dWV": r["dWV"]}

@@ -471,3 +471,86 @@ def test_planted_softmax_without_max_shift_still_exact_but_lse_wrong(monkeypatch
         return e / tot, np.log(tot)[:, 0] + 1e-9
     monkeypatch.setattr(ra, "softmax_rows", bad)
     assert _broken(_all_pins())
+
+
+# ---------------------------------------------------------------------------------------
+# One combined weight X (the page's own parameterisation dLoss/dx = A~^T vec(gamma))
+# ---------------------------------------------------------------------------------------
+
+def _tiny_x(n, d, seed=0, B=1, H=1):
+    inp = _tiny(n, d, H=H, B=B, seed=seed)
+    rng = np.random.default_rng(seed + 100)
+    inp["X"] = rng.standard_normal((H, d, d)) / math.sqrt(d)
+    return inp
+
+
+def test_rotation_matrix_matches_rope_and_composes():
+    rng = np.random.default_rng(4)
+    d = 6
+    a, b = rng.uniform(-3, 3, d // 2), rng.uniform(-3, 3, d // 2)
+    Ra, Rb = ra.rotation_matrix(a), ra.rotation_matrix(b)
+    x = rng.standard_normal(d)
+    assert np.allclose(Ra @ x, ra.rope_rotate(x[None, :], a[None, :])[0], atol=1e-14)
+    assert np.allclose(Ra.T @ Ra, np.eye(d), atol=1e-14)
+    assert np.allclose(Ra @ Rb, ra.rotation_matrix(a + b), atol=1e-13)
+
+
+@pytest.mark.parametrize("n,d", [(1, 2), (3, 2), (4, 4), (6, 4)])
+@pytest.mark.parametrize("causal", [False, True])
+def test_combined_weight_literal_finite_differences(n, d, causal):
+    """A~^T vec(gamma), built literally row by row, against central differences of the loss."""
+    inp = _tiny_x(n, d, seed=n + d)
+    args = lambda X: (inp["A1"][0, 0], inp["A2"][0, 0], inp["A3"][0, 0], inp["E"][0, 0], X,
+                      inp["WV"][0], inp["pos"], causal, 10.0)
+    X = inp["X"][0].copy()
+    g = ra.combined_weight_literal(*args(X))["dX"]
+    fd = np.zeros_like(X)
+    for idx in np.ndindex(X.shape):
+        step = 1e-5 * max(1.0, abs(X[idx]))
+        Xp, Xm = X.copy(), X.copy()
+        Xp[idx] += step
+        Xm[idx] -= step
+        fd[idx] = (ra.combined_weight_literal(*args(Xp))["loss"]
+                   - ra.combined_weight_literal(*args(Xm))["loss"]) / (2 * step)
+    assert _rel(g, fd) <= 1e-6
+
+
+def combined_route_error(inp, causal, base):
+    """max relative difference between the literal A~^T vec(gamma) form and the general
+    problem with WQ = I, WK = X^T (loss, dX, dWV) over the instances of ``inp``."""
+    eff = oracle.combined_weight_forward_backward(inp, causal, base)
+    B, H = inp["A1"].shape[:2]
+    worst = 0.0
+    dX_sum = np.zeros_like(eff["dX"])
+    dWV_sum = np.zeros_like(eff["dWV"])
+    loss = 0.0
+    for b in range(B):
+        for h in range(H):
+            lit = ra.combined_weight_literal(inp["A1"][b, h], inp["A2"][b, h], inp["A3"][b, h],
+                                             inp["E"][b, h], inp["X"][h], inp["WV"][h],
+                                             inp["pos"], causal, base)
+            dX_sum[h] += lit["dX"]
+            dWV_sum[h] += lit["dWV"]
+            loss += lit["loss"]
+    worst = max(worst, _rel(eff["dX"], dX_sum), _rel(eff["dWV"], dWV_sum),
+                abs(eff["loss"] - loss) / abs(loss))
+    return worst
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_combined_weight_literal_equals_general_route(causal):
+    inp = _tiny_x(5, 4, seed=8, B=2, H=2)
+    inp["pos"] = np.array([3, 7, 8, 20, 21], dtype=np.int32)   # non-contiguous positions
+    assert combined_route_error(inp, causal, 1e4) <= 1e-12
+
+
+def test_planted_combined_weight_missing_transpose(monkeypatch):
+    """dX taken as dWK instead of dWK^T breaks the literal-vs-general pin."""
+    orig = oracle.combined_weight_forward_backward
+
+    def bad(inp, causal, base):
+        out = orig(inp, causal, base)
+        out["dX"] = np.transpose(out["dX"], (0, 2, 1))
+        return out
+    monkeypatch.setattr(oracle, "combined_weight_forward_backward", bad)
+    assert combined_route_error(_tiny_x(4, 4, seed=3), False, 10.0) > 1e-3
