@@ -122,6 +122,22 @@ ra_status rope_attn_loss_bwd_inputs(const ra_problem* p, const void* O, const fl
                                     int32_t ws_holds_fwd, void* stream);
 
 /*
+ * One combined weight per head, the parameterisation of the page's problem: the gradient with
+ * respect to a single weight x, dLoss/dx = A~^T vec(gamma(x)) ("RoPE Attention kan bijna lineair
+ * worden getraind", Probleemdefinitie and Methodologie 1), read as x = vec(X) in the score
+ *   z_ij = a1_i^T R_{j-i} X a2_j / sqrt(d)      (R_{j-i}: RoPE rotation by pos_j - pos_i).
+ * Since R_{j-i} = R_i^T R_j, this is the general problem with WQ = I and WK = X^T:
+ *   rope_attn_combined_weights writes WQ = I and WK = X^T ([H][d][d], element type `dtype`) for
+ *   a following rope_attn_fwd / rope_attn_loss_bwd, and rope_attn_combined_grad turns that
+ *   call's dWK (fp32 [H][d][d]) into dX = dWK^T (fp32 [H][d][d]).
+ * X, WQ, WK, dWK, dX: device, 16-byte aligned; d in {64, 128}; H >= 1.  Errors as above.
+ */
+ra_status rope_attn_combined_weights(const void* X, int32_t H, int32_t d, int32_t dtype,
+                                     void* WQ, void* WK, void* stream);
+ra_status rope_attn_combined_grad(const float* dWK, int32_t H, int32_t d, float* dX,
+                                  void* stream);
+
+/*
  * Synchronises `stream`, then reports and clears the device-side status word of the current
  * device: RA_ERR_TIMEOUT if a kernel gave up waiting since the last call, else RA_OK
  * (RA_ERR_CUDA if the synchronisation itself failed).

@@ -42,13 +42,15 @@ enum KernelId : int {
   K_DW_TC,
   K_DA_TC,
   K_DA_SIMT,
+  K_COMB_W,
+  K_COMB_G,
   K_COUNT
 };
 const char* const kKernelNames[K_COUNT] = {
     "rope_table", "proj_rope_simt", "attn_fwd_simt", "bwd_pre",
     "attn_bwd_simt", "dw_partial_simt", "dw_reduce", "loss_finalize",
     "attn_fwd_tc", "attn_bwd_tc", "proj_rope_tc", "dq_unrotate", "dw_tc",
-    "input_grads_tc", "input_grads_simt"};
+    "input_grads_tc", "input_grads_simt", "combined_weights", "combined_grad"};
 
 struct ProfRecord {
   int id;
@@ -741,6 +743,36 @@ ra_status rope_attn_loss_bwd_inputs(const ra_problem* p, const void* O, const fl
   if (p->dtype == RA_F32) return simt_input_grads(p, L, dA1, dA2, dA3, ws, st);
   return p->d == 128 ? tc_input_grads<128>(p, L, dA1, dA2, dA3, ws, st)
                      : tc_input_grads<64>(p, L, dA1, dA2, dA3, ws, st);
+}
+
+ra_status rope_attn_combined_weights(const void* X, int32_t H, int32_t d, int32_t dtype,
+                                     void* WQ, void* WK, void* stream) {
+  if (!X || !WQ || !WK || H < 1 || (d != 64 && d != 128)) return RA_ERR_INVALID_ARG;
+  if (dtype != RA_F32 && dtype != RA_BF16) return RA_ERR_INVALID_ARG;
+  if (!is_aligned(X, 16) || !is_aligned(WQ, 16) || !is_aligned(WK, 16)) return RA_ERR_ALIGNMENT;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const long long total = (long long)H * d * d;
+  const unsigned blocks = (unsigned)((total + 255) / 256);
+  Launch l(K_COMB_W, st);
+  if (dtype == RA_F32)
+    ra::simt::combined_weights_kernel<float><<<blocks, 256, 0, st>>>(
+        (const float*)X, (float*)WQ, (float*)WK, total, d);
+  else
+    ra::simt::combined_weights_kernel<__nv_bfloat16><<<blocks, 256, 0, st>>>(
+        (const __nv_bfloat16*)X, (__nv_bfloat16*)WQ, (__nv_bfloat16*)WK, total, d);
+  return launch_status();
+}
+
+ra_status rope_attn_combined_grad(const float* dWK, int32_t H, int32_t d, float* dX,
+                                  void* stream) {
+  if (!dWK || !dX || H < 1 || (d != 64 && d != 128)) return RA_ERR_INVALID_ARG;
+  if (!is_aligned(dWK, 16) || !is_aligned(dX, 16)) return RA_ERR_ALIGNMENT;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const long long total = (long long)H * d * d;
+  Launch l(K_COMB_G, st);
+  ra::simt::transpose_heads_kernel<<<(unsigned)((total + 255) / 256), 256, 0, st>>>(
+      dWK, dX, total, d);
+  return launch_status();
 }
 
 ra_status rope_attn_step_noalloc(const ra_problem* p, void* O, float* lse, float* loss,

@@ -513,5 +513,29 @@ input_grad_kernel(const float* __restrict__ dQt, const float* __restrict__ dKt,
   }
 }
 
+// ---------------------------------------------------------------------------------------
+// One combined weight X per head: WQ = I and WK = X^T make the general problem's scores
+// q~_i . k~_j = a1_i^T R_{j-i} X a2_j; its dWK is then dX^T.
+// ---------------------------------------------------------------------------------------
+template <class T>
+__global__ void combined_weights_kernel(const T* __restrict__ X, T* __restrict__ WQ,
+                                        T* __restrict__ WK, long long total, int d) {
+  const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= total) return;
+  const long long hd = idx / ((long long)d * d);
+  const int rc = (int)(idx - hd * d * d), r = rc / d, c = rc - r * d;
+  WQ[idx] = from_f<T>(r == c ? 1.f : 0.f);
+  WK[idx] = X[hd * d * d + (long long)c * d + r];
+}
+
+__global__ void transpose_heads_kernel(const float* __restrict__ in, float* __restrict__ out,
+                                       long long total, int d) {
+  const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= total) return;
+  const long long hd = idx / ((long long)d * d);
+  const int rc = (int)(idx - hd * d * d), r = rc / d, c = rc - r * d;
+  out[idx] = in[hd * d * d + (long long)c * d + r];
+}
+
 }  // namespace simt
 }  // namespace ra

@@ -21,7 +21,8 @@ RA_F32, RA_BF16 = 0, 1
 EXPORTED = ("rope_attn_workspace_bytes", "rope_attn_fwd", "rope_attn_loss_bwd",
             "rope_attn_last_error", "rope_attn_status_string", "rope_attn_launch_count",
             "rope_attn_profile_enable", "rope_attn_profile_read", "rope_attn_kernel_name",
-            "rope_attn_step_noalloc", "rope_attn_loss_bwd_inputs")
+            "rope_attn_step_noalloc", "rope_attn_loss_bwd_inputs", "rope_attn_combined_weights",
+            "rope_attn_combined_grad")
 
 # Capacity of the static scratch behind rope_attn_step_noalloc (RA_NOALLOC_SCRATCH_BYTES).
 NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
@@ -82,6 +83,10 @@ def load() -> ctypes.CDLL:
     lib.rope_attn_loss_bwd_inputs.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz,
                                               i32, vp]
     lib.rope_attn_loss_bwd_inputs.restype = ctypes.c_int
+    lib.rope_attn_combined_weights.argtypes = [vp, i32, i32, i32, vp, vp, vp]
+    lib.rope_attn_combined_weights.restype = ctypes.c_int
+    lib.rope_attn_combined_grad.argtypes = [vp, i32, i32, vp, vp]
+    lib.rope_attn_combined_grad.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -162,6 +167,25 @@ def loss_bwd_inputs(prob: Problem, O, lse, loss, dWQ, dWK, dWV, dA1, dA2, dA3, w
         int(bool(ws_holds_fwd)), _stream(stream))
     if st != RA_OK:
         raise RopeAttnError(st, "rope_attn_loss_bwd_inputs")
+
+
+def combined_weights(X, WQ, WK, stream=None) -> None:
+    """rope_attn_combined_weights: WQ = I, WK = X^T per head (X, WQ, WK: [H][d][d])."""
+    import torch
+    H, d = X.shape[0], X.shape[1]
+    dt = RA_F32 if X.dtype == torch.float32 else RA_BF16
+    st = load().rope_attn_combined_weights(_ptr(X), H, d, dt, _ptr(WQ), _ptr(WK),
+                                           _stream(stream))
+    if st != RA_OK:
+        raise RopeAttnError(st, "rope_attn_combined_weights")
+
+
+def combined_grad(dWK, dX, stream=None) -> None:
+    """rope_attn_combined_grad: dX = dWK^T per head (fp32 [H][d][d])."""
+    H, d = dWK.shape[0], dWK.shape[1]
+    st = load().rope_attn_combined_grad(_ptr(dWK), H, d, _ptr(dX), _stream(stream))
+    if st != RA_OK:
+        raise RopeAttnError(st, "rope_attn_combined_grad")
 
 
 def step_noalloc(prob: Problem, O, lse, loss, dWQ, dWK, dWV, stream=None) -> None:
@@ -259,3 +283,30 @@ class RopeAttention:
     def step(self, stream=None):
         self.forward(stream)
         return self.backward(True, stream)
+
+
+class RopeAttentionX:
+    """The page's parameterisation: one combined weight X per head (score
+    a1_i^T R_{j-i} X a2_j / sqrt(d)) and the value weight WV.  ``step()`` returns
+    (loss, dX, dWV) as device tensors; call ``set_weights(X)`` after changing X."""
+
+    def __init__(self, A1, A2, A3, X, WV, E, pos=None, causal=False, rope_base=10000.0):
+        import torch
+        H, d = X.shape[0], X.shape[1]
+        self.WQ = torch.empty_like(X)
+        self.WK = torch.empty_like(X)
+        combined_weights(X, self.WQ, self.WK)
+        self.attn = RopeAttention(A1, A2, A3, self.WQ, self.WK, WV, E, pos, causal, rope_base)
+        self.dX = torch.empty((H, d, d), dtype=torch.float32, device=X.device)
+
+    def set_weights(self, X, stream=None):
+        combined_weights(X, self.WQ, self.WK, stream)
+
+    def forward(self, stream=None):
+        return self.attn.forward(stream)
+
+    def step(self, stream=None):
+        self.attn.forward(stream)
+        self.attn.backward(True, stream)
+        combined_grad(self.attn.dWK, self.dX, stream)
+        return self.attn.loss, self.dX, self.attn.dWV
