@@ -265,8 +265,10 @@ class RopeAttention:
         return self.O, self.lse, self.loss
 
     def backward(self, ws_holds_fwd=True, stream=None):
-        loss_bwd(self.prob, self.O, self.lse, self.loss, self.dWQ, self.dWK, self.dWV, self.ws,
-                 ws_holds_fwd, stream)
+        # after this object's forward the loss is already in self.loss: the backward need not
+        # sum the partials again
+        loss_bwd(self.prob, self.O, self.lse, None if ws_holds_fwd else self.loss, self.dWQ,
+                 self.dWK, self.dWV, self.ws, ws_holds_fwd, stream)
         return self.loss, self.dWQ, self.dWK, self.dWV
 
     def backward_inputs(self, ws_holds_fwd=True, stream=None):
@@ -276,8 +278,9 @@ class RopeAttention:
             self.dA1 = torch.empty_like(self.O)
             self.dA2 = torch.empty_like(self.O)
             self.dA3 = torch.empty_like(self.O)
-        loss_bwd_inputs(self.prob, self.O, self.lse, self.loss, self.dWQ, self.dWK, self.dWV,
-                        self.dA1, self.dA2, self.dA3, self.ws, ws_holds_fwd, stream)
+        loss_bwd_inputs(self.prob, self.O, self.lse, None if ws_holds_fwd else self.loss,
+                        self.dWQ, self.dWK, self.dWV, self.dA1, self.dA2, self.dA3, self.ws,
+                        ws_holds_fwd, stream)
         return self.loss, self.dWQ, self.dWK, self.dWV, self.dA1, self.dA2, self.dA3
 
     def step(self, stream=None):
