@@ -110,6 +110,42 @@ def test_bwd_argument_errors():
     assert _bwd(p, nbytes=nb - 256) == ra.RA_ERR_WORKSPACE
 
 
+def test_bwd_inputs_argument_errors():
+    """rope_attn_loss_bwd_inputs validates its extra outputs, then everything the plain
+    backward validates, before anything is launched."""
+    lib = ra.load()
+    p = _prob()
+    nb = lib.rope_attn_workspace_bytes(ctypes.byref(p))
+
+    def call(prob=p, dA=(FAKE, FAKE, FAKE), nbytes=nb, holds=1, O=FAKE):
+        return lib.rope_attn_loss_bwd_inputs(ctypes.byref(prob), O, FAKE, FAKE, FAKE, FAKE,
+                                             FAKE, *dA, FAKE * 16, nbytes, holds, None)
+    assert call(dA=(None, FAKE, FAKE)) == ra.RA_ERR_INVALID_ARG
+    assert call(dA=(FAKE, FAKE, None)) == ra.RA_ERR_INVALID_ARG
+    assert call(dA=(FAKE, FAKE + 8, FAKE)) == ra.RA_ERR_ALIGNMENT
+    assert call(prob=_prob(E=None)) == ra.RA_ERR_INVALID_ARG
+    assert call(O=None) == ra.RA_ERR_INVALID_ARG
+    assert call(holds=3) == ra.RA_ERR_INVALID_ARG
+    assert call(nbytes=nb - 256) == ra.RA_ERR_WORKSPACE
+
+
+def test_combined_weight_argument_errors():
+    lib = ra.load()
+    w = lambda X=FAKE, H=2, d=64, dt=ra.RA_BF16, WQ=FAKE, WK=FAKE: \
+        lib.rope_attn_combined_weights(X, H, d, dt, WQ, WK, None)
+    assert w(X=None) == ra.RA_ERR_INVALID_ARG
+    assert w(WK=None) == ra.RA_ERR_INVALID_ARG
+    assert w(H=0) == ra.RA_ERR_INVALID_ARG
+    assert w(d=32) == ra.RA_ERR_INVALID_ARG
+    assert w(dt=5) == ra.RA_ERR_INVALID_ARG
+    assert w(WQ=FAKE + 4) == ra.RA_ERR_ALIGNMENT
+    g = lambda dWK=FAKE, H=2, d=128, dX=FAKE: lib.rope_attn_combined_grad(dWK, H, d, dX, None)
+    assert g(dWK=None) == ra.RA_ERR_INVALID_ARG
+    assert g(H=-1) == ra.RA_ERR_INVALID_ARG
+    assert g(d=96) == ra.RA_ERR_INVALID_ARG
+    assert g(dX=FAKE + 8) == ra.RA_ERR_ALIGNMENT
+
+
 def test_status_strings():
     for s in range(7):
         assert ra.status_string(s).startswith("RA_")
