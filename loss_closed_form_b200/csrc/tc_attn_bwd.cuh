@@ -331,12 +331,15 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     if (ok) ok = mbar_wait_warp(b_acc, 0, abort_flag, lim);
     const uint32_t tab_s = sbase + C::K_OFF;
     const uint32_t stg = sbase + C::Q_OFF + half * C::KTILE;
-    if (ok && tid == 0) {
+    const bool tab_issued = ok && tid == 0;
+    if (tab_issued) {
       mbar_expect_tx(b_tab, C::TABT);
       for (int b = 0; b < D / 32; ++b)
         tma_load_2d(tab_s + b * C::TBLK, &tm_tab, b_tab, 32 * b, kt * C::BK);
     }
     if (ok && half == 0) ok = mbar_wait_warp(b_tab, 0, abort_flag, lim);
+    // after an abort, the copy this thread issued lands before the CTA leaves
+    if (tab_issued && !ok) mbar_drain(b_tab, 0, lim);
     if (ok) {
       tc_fence_after();
       const uint32_t src = tmem + lane_base + (half == 0 ? C::T_DK : C::T_DV);

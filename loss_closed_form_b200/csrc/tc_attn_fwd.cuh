@@ -350,12 +350,15 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
     const bool vrow = row < n;
     const uint32_t stg = sbase + C::Q_OFF + t * C::TILE;
     const bool has_e = p.E != nullptr;
-    if (ok && r == 0 && has_e) {
+    const bool e_issued = ok && r == 0 && has_e;
+    if (e_issued) {
       mbar_expect_tx(b_efull(t), C::TILE);
       for (int b = 0; b < C::KB; ++b)
         tma_load_3d(stg + b * C::BLK, &tm_e, b_efull(t), 64 * b, qt * C::BM, bh);
     }
     if (ok && has_e) ok = mbar_wait_warp(b_efull(t), 0, abort_flag, lim);
+    // after an abort, the copy this thread issued lands before the CTA leaves
+    if (e_issued && !ok) mbar_drain(b_efull(t), 0, lim);
     uint32_t lw[D / 2];  // l = O - E of this row, bf16 pairs
     if (ok) {
       tc_fence_after();
