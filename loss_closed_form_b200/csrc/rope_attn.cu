@@ -456,7 +456,8 @@ ra_status tc_weight_grads(const ra_problem* p, const Layout& L, float* dWQ, floa
     const long long quads = (long long)BH * n * (half / 4);
     Launch l(K_DQ_UNROT, st);
     dq_unrotate_kernel<<<(unsigned)((quads + 255) / 256), 256, 0, st>>>(
-        at<float4>(ws, L.dqt), at<float4>(ws, L.rope), at<uint4>(ws, L.dq16), quads, n, half);
+        at<float4>(ws, L.dqt), at<float4>(ws, L.rope), at<uint4>(ws, L.dq16), quads, n, half,
+        1.0f / sqrtf((float)D));
   }
   CUtensorMap a1, a2, a3, x1, x2, x3;
   if (!map_bf16_3d(&a1, p->A1, D, n, BH, C::BR) || !map_bf16_3d(&a2, p->A2, D, n, BH, C::BR) ||

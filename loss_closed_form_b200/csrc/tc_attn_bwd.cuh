@@ -12,7 +12,10 @@
 //   dV    += P^T l_i                   (accumulated in TMEM over all query tiles)
 //   dK~   += gamma^T Q~_i              (scaled by 1/sqrt(d) and un-rotated at the end)
 //   dQ~_i^T = K~^T gamma^T             (d on TMEM lanes; staged in shared memory and added to
-//                                        the global fp32 dQ~ by one TMA bulk reduce-add)
+//                                        the global fp32 accumulator by one TMA bulk
+//                                        reduce-add; the 1/sqrt(d) is applied when the
+//                                        accumulator is un-rotated, which keeps the drain warps'
+//                                        per-element work to a load and a store)
 // so no n x n matrix ever leaves the chip.
 //
 // Definitions: "RoPE Attention kan bijna lineair worden getraind", Methodologie 1 (s, l,
@@ -407,8 +410,8 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         // row-major [q][d] fp32: for one q the lanes write consecutive d
 #pragma unroll
         for (int c = 0; c < 32; ++c) {
-          st_shared_f32(stage + (c * D + drow) * 4, __uint_as_float(r0[c]) * p.scale);
-          st_shared_f32(stage + ((32 + c) * D + drow) * 4, __uint_as_float(r1[c]) * p.scale);
+          st_shared_f32(stage + (c * D + drow) * 4, __uint_as_float(r0[c]));
+          st_shared_f32(stage + ((32 + c) * D + drow) * 4, __uint_as_float(r1[c]));
         }
       }
       fence_proxy_async_smem();

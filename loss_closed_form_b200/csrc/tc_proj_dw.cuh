@@ -2,7 +2,7 @@
 //
 //   proj_rope_tc: X = A_z W_z for a 128-row tile (tcgen05, A K-major, W as an MN-major B),
 //                 then RoPE on (2k, 2k+1) pairs for Q and K in the epilogue, bf16 out.
-//   dq_unrotate:  dQ = rot^-1(dQ~) (fp32 accumulator in, bf16 out).
+//   dq_unrotate:  dQ = rot^-1(acc) / sqrt(d) (fp32 accumulator of gamma K~ in, bf16 out).
 //   dw_tc:        dW_z[h] partial = sum over a range of 128-row tiles of A_z^T dX_z
 //                 (both operands MN-major; fp32 partials reduced in a fixed order later).
 //
@@ -260,12 +260,13 @@ proj_rope_tc_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_cons
 }
 
 // ---------------------------------------------------------------------------------------
-// dQ = rot^-1(dQ~): fp32 in, bf16 out; one thread per four pairs (d/2 is a multiple of 4,
+// dQ = rot^-1(acc) / sqrt(d): fp32 in, bf16 out; one thread per four pairs (d/2 is a multiple of 4,
 // so the four pairs share a row): two 16-byte loads of dQ~ and of (cos, sin), one 16-byte
 // store.
 // ---------------------------------------------------------------------------------------
 __global__ void dq_unrotate_kernel(const float4* __restrict__ dqt, const float4* __restrict__ tab,
-                                   uint4* __restrict__ dq, long long quads, int n, int half) {
+                                   uint4* __restrict__ dq, long long quads, int n, int half,
+                                   float scale) {
   const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (idx >= quads) return;
   const int qpr = half / 4;  // quads per row
@@ -275,8 +276,9 @@ __global__ void dq_unrotate_kernel(const float4* __restrict__ dqt, const float4*
   const float4 y0 = dqt[2 * idx], y1 = dqt[2 * idx + 1];
   const float4* tr = tab + ((size_t)i * half) / 2 + 2 * k;
   const float4 c0 = tr[0], c1 = tr[1];
-  auto rot = [](float x, float y, float c, float sn) {
-    return pack_bf16x2(x * c + y * sn, -x * sn + y * c);
+  // the accumulator holds gamma K~ summed over key tiles: scale by 1/sqrt(d), rotate by -phi
+  auto rot = [scale](float x, float y, float c, float sn) {
+    return pack_bf16x2((x * c + y * sn) * scale, (-x * sn + y * c) * scale);
   };
   dq[idx] = make_uint4(rot(y0.x, y0.y, c0.x, c0.y), rot(y0.z, y0.w, c0.z, c0.w),
                        rot(y1.x, y1.y, c1.x, c1.y), rot(y1.z, y1.w, c1.z, c1.w));
