@@ -207,22 +207,23 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       constexpr uint32_t idesc_sb = idesc_bf16_f32(128, C::BQ, false, false);
       constexpr uint32_t idesc_kv = idesc_bf16_f32(128, D, false, true);
       constexpr uint32_t idesc_dq = idesc_bf16_f32(D, C::BQ, true, true);
-      const uint32_t ka = sbase + C::K_OFF, va = sbase + C::V_OFF;
+      // descriptor low words per buffer (sw128_lo), offsets added per K step (sw128_at)
+      const uint32_t ka_k = sw128_lo(sbase + C::K_OFF, 16), va_k = sw128_lo(sbase + C::V_OFF, 16);
+      const uint32_t ka_mn = sw128_lo(sbase + C::K_OFF, C::KBLK);
+      const uint32_t gt_mn = sw128_lo(sbase + C::G_OFF, C::KBLK);
       bool ok = mbar_wait(b_kv, 0, abort_flag, lim);
       auto issue_sb = [&](int ii) -> bool {
         const int s = ii % C::NSQ;
         if (!mbar_wait(b_qfull(s), (ii / C::NSQ) & 1, abort_flag, lim)) return false;
         tc_fence_after();
-        const uint32_t qb = sbase + C::Q_OFF + s * C::QTILE;
-        const uint32_t lb = sbase + C::L_OFF + s * C::QTILE;
+        const uint32_t qb_k = sw128_lo(sbase + C::Q_OFF + s * C::QTILE, 16);
+        const uint32_t lb_k = sw128_lo(sbase + C::L_OFF + s * C::QTILE, 16);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t ko = (kk >> 2) * C::KBLK + (kk & 3) * 32;
           const uint32_t qo = (kk >> 2) * C::QBLK + (kk & 3) * 32;
-          mma_ss(tmem + C::T_S, sw128_desc(ka + ko, 16, 1024), sw128_desc(qb + qo, 16, 1024),
-                 idesc_sb, kk > 0);
-          mma_ss(tmem + C::T_B, sw128_desc(va + ko, 16, 1024), sw128_desc(lb + qo, 16, 1024),
-                 idesc_sb, kk > 0);
+          mma_ss(tmem + C::T_S, sw128_at(ka_k, ko), sw128_at(qb_k, qo), idesc_sb, kk > 0);
+          mma_ss(tmem + C::T_B, sw128_at(va_k, ko), sw128_at(lb_k, qo), idesc_sb, kk > 0);
         }
         mma_commit(b_sfull);
         return true;
@@ -237,17 +238,16 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         const int s = ii % C::NSQ;
         if (!(ok = mbar_wait(b_pgfull, ii & 1, abort_flag, lim))) break;
         tc_fence_after();
-        const uint32_t gt = sbase + C::G_OFF;
-        const uint32_t qb = sbase + C::Q_OFF + s * C::QTILE;
-        const uint32_t lb = sbase + C::L_OFF + s * C::QTILE;
+        const uint32_t qb_mn = sw128_lo(sbase + C::Q_OFF + s * C::QTILE, C::QBLK);
+        const uint32_t lb_mn = sw128_lo(sbase + C::L_OFF + s * C::QTILE, C::QBLK);
         // dV += P^T l_i, dK += gamma^T Q~_i: M = 128 keys, N = D, K = 64 queries, with
         // P^T and gamma^T read from TMEM (two bf16 per column, 8 columns per K step)
 #pragma unroll
         for (int kk = 0; kk < C::BQ / 16; ++kk) {
-          mma_ts(tmem + C::T_DV, tmem + C::T_PT + kk * 8,
-                 sw128_desc(lb + kk * 2048, C::QBLK, 1024), idesc_kv, (ii > 0 || kk > 0));
-          mma_ts(tmem + C::T_DK, tmem + C::T_GT + kk * 8,
-                 sw128_desc(qb + kk * 2048, C::QBLK, 1024), idesc_kv, (ii > 0 || kk > 0));
+          mma_ts(tmem + C::T_DV, tmem + C::T_PT + kk * 8, sw128_at(lb_mn, kk * 2048), idesc_kv,
+                 (ii > 0 || kk > 0));
+          mma_ts(tmem + C::T_DK, tmem + C::T_GT + kk * 8, sw128_at(qb_mn, kk * 2048), idesc_kv,
+                 (ii > 0 || kk > 0));
         }
         // dQ~_i^T = K~^T gamma^T   (M = D, N = 64 queries, K = 128 keys), once the drain has
         // read the previous tile's dQ~ out of TMEM
@@ -257,8 +257,8 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         }
 #pragma unroll
         for (int kk = 0; kk < C::BK / 16; ++kk)
-          mma_ss(tmem + C::T_DQ, sw128_desc(ka + kk * 2048, C::KBLK, 1024),
-                 sw128_desc(gt + kk * 2048, C::KBLK, 1024), idesc_dq, kk > 0);
+          mma_ss(tmem + C::T_DQ, sw128_at(ka_mn, kk * 2048), sw128_at(gt_mn, kk * 2048),
+                 idesc_dq, kk > 0);
         mma_commit(b_dqfull);
         mma_commit(b_pgfree);
         mma_commit(b_qempty(s));

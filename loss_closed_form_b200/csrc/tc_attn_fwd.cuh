@@ -190,25 +190,25 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, false, false);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, false, true);
       const uint32_t qa0 = sbase + C::Q_OFF;
+      // descriptor low words per buffer (sw128_lo), offsets added per K step (sw128_at)
       auto issue_s = [&](int t, int j) {
-        const uint32_t qa = qa0 + t * C::TILE;
-        const uint32_t kb = sbase + C::K_OFF + (j % C::NS) * C::TILE;
+        const uint32_t qa = sw128_lo(qa0 + t * C::TILE, 16);
+        const uint32_t kb = sw128_lo(sbase + C::K_OFF + (j % C::NS) * C::TILE, 16);
         const uint32_t d_s = tmem + C::T_S0 + 128 * t;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * C::BLK + (kk & 3) * 32;
-          mma_ss(d_s, sw128_desc(qa + off, 16, 1024), sw128_desc(kb + off, 16, 1024), idesc_s,
-                 kk > 0);
+          mma_ss(d_s, sw128_at(qa, off), sw128_at(kb, off), idesc_s, kk > 0);
         }
         mma_commit(b_sfull(t));
       };
       auto issue_pv = [&](int t, int j) {
         const uint32_t pa = tmem + C::T_S0 + 128 * t;
-        const uint32_t vb = sbase + C::V_OFF + (j % C::NS) * C::TILE;
+        const uint32_t vb = sw128_lo(sbase + C::V_OFF + (j % C::NS) * C::TILE, C::BLK);
 #pragma unroll
         for (int kk = 0; kk < C::BN / 16; ++kk)
-          mma_ts(tmem + C::T_O0 + 128 * t, pa + kk * 8, sw128_desc(vb + kk * 2048, C::BLK, 1024),
-                 idesc_pv, (j > 0 || kk > 0));
+          mma_ts(tmem + C::T_O0 + 128 * t, pa + kk * 8, sw128_at(vb, kk * 2048), idesc_pv,
+                 (j > 0 || kk > 0));
         mma_commit(b_pvdone(t));
       };
       bool ok = mbar_wait(b_q, 0, abort_flag, lim);

@@ -251,6 +251,17 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr, uint32_t lbo, uin
   return d;
 }
 
+// The same descriptor split for issue loops: sw128_lo(base, lbo) once per buffer, then
+// sw128_at(lo, off) for a constant byte offset off inside it (one integer add: the start
+// field is address >> 4 and shared addresses stay below 2^18, so no carry leaves it).
+__device__ __forceinline__ uint32_t sw128_lo(uint32_t saddr, uint32_t lbo) {
+  return ((saddr >> 4) & 0x3FFFu) | (((lbo >> 4) & 0x3FFFu) << 16);
+}
+__device__ __forceinline__ uint64_t sw128_at(uint32_t lo, uint32_t off) {
+  constexpr uint32_t hi = (1024u >> 4) | (1u << 14) | (2u << 29);  // SBO 1024, v1, 128B swizzle
+  return (static_cast<uint64_t>(hi) << 32) | (lo + (off >> 4));
+}
+
 // Instruction descriptor, kind::f16 with bf16 A and B, fp32 accumulator.
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn_major,
                                                       bool b_mn_major) {
