@@ -271,14 +271,17 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
     for (int j = 0; j < Tt; ++j) {
       if (!(ok = mbar_wait_warp(b_sfull(t), j & 1, abort_flag, lim))) break;
       tc_fence_after();
+      // the four 32-column loads share one wait
+      uint32_t xr[4][32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld32(s_col + 32 * c, xr[c]);
+      tmem_wait_ld();
       float x[128];
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
-        uint32_t rr[32];
-        tmem_ld32(s_col + 32 * c, rr);
-        tmem_wait_ld();
+        reg_fence32(xr[c]);
 #pragma unroll
-        for (int i = 0; i < 32; ++i) x[32 * c + i] = __uint_as_float(rr[i]);
+        for (int i = 0; i < 32; ++i) x[32 * c + i] = __uint_as_float(xr[c][i]);
       }
       const int key0 = j * C::BN;
       if (key0 + C::BN > n || (p.causal && j == qt)) {
@@ -288,15 +291,18 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
           if (key >= n || (p.causal && key > row)) x[i] = -INFINITY;
         }
       }
-      float mt0 = x[0], mt1 = x[1], mt2 = x[2], mt3 = x[3];
+      // row maximum: four chains of three-input max (elements k, k + 4, k + 8, ...)
+      float mt[4];
 #pragma unroll
-      for (int i = 4; i < 128; i += 4) {
-        mt0 = fmaxf(mt0, x[i]);
-        mt1 = fmaxf(mt1, x[i + 1]);
-        mt2 = fmaxf(mt2, x[i + 2]);
-        mt3 = fmaxf(mt3, x[i + 3]);
+      for (int k = 0; k < 4; ++k) mt[k] = fmax3f(x[k], x[k + 4], x[k + 8]);
+#pragma unroll
+      for (int i = 12; i < 124; i += 8) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) mt[k] = fmax3f(mt[k], x[i + k], x[i + 4 + k]);
       }
-      const float mnew = fmaxf(m, fmaxf(fmaxf(mt0, mt1), fmaxf(mt2, mt3)) * p.scale_log2);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) mt[k] = fmaxf(mt[k], x[124 + k]);
+      const float mnew = fmaxf(m, fmax3f(mt[0], mt[1], fmaxf(mt[2], mt[3])) * p.scale_log2);
       if (j == 0) {
         m = mnew;
       } else {
