@@ -125,7 +125,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(b_sfull(t), 1);
-      mbar_init(b_pfull(t), 128);
+      mbar_init(b_pfull(t), 4);  // one arrival per softmax warp
       mbar_init(b_pvdone(t), 1);
     }
     mbar_init(b_drain, 1);
@@ -343,7 +343,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
       l += ps0 + ps1;
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(b_pfull(t));
+      mbar_arrive_warp(b_pfull(t));
     }
     // ---- epilogue: one full row of O per thread.  The tile's query buffer is free (every
     //      S_t has completed): E_t comes in there by TMA, each thread overwrites its own row
