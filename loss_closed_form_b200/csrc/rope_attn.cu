@@ -210,6 +210,15 @@ int num_sms() {
   return v;
 }
 
+// Heads per scheduling group of the attention kernels: as many as keep the tensors that
+// every CTA of a head re-reads (bytes_per_head) within about half of the 126 MB L2, at
+// least one.
+constexpr double kL2GroupBytes = 64.0 * 1024 * 1024;
+int heads_per_l2_group(double bytes_per_head, int BH) {
+  const int g = static_cast<int>(kL2GroupBytes / bytes_per_head);
+  return g < 1 ? 1 : (g > BH ? BH : g);
+}
+
 ra_status launch_status() {
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? RA_OK : RA_ERR_CUDA;
@@ -517,11 +526,12 @@ ra_status tc_fwd_launch(const ra_problem* p, const Layout& L, void* O, float* ls
   fp.nq = (n + C::BM - 1) / C::BM;
   fp.npair = (fp.nq + 1) / 2;
   fp.causal = p->causal;
+  fp.hgroup = heads_per_l2_group(4.0 * n * D, BH);  // K~ and V, bf16
   fp.scale_log2 = ra::kLog2e / sqrtf((float)D);
   fp.limit_ns = wait_limit_ns();
   auto k = attn_fwd_tc_kernel<D>;
   cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_ALLOC);
-  dim3 grid(fp.npair, BH);
+  dim3 grid(fp.hgroup, fp.npair, (BH + fp.hgroup - 1) / fp.hgroup);
   Launch l(K_FWD_TC, st);
   k<<<grid, C::THREADS, C::SMEM_ALLOC, st>>>(mq, mk, mv, me, mo, mell, fp);
   return RA_OK;
@@ -566,12 +576,13 @@ ra_status tc_bwd_launch(const ra_problem* p, const Layout& L, const float* lse, 
   bp.BH = BH;
   bp.nk = (n + C::BK - 1) / C::BK;
   bp.causal = p->causal;
+  bp.hgroup = heads_per_l2_group(8.0 * n * D, BH);  // Q~, l (bf16) and dQ~ (fp32)
   bp.scale = 1.0f / sqrtf((float)D);
   bp.scale_log2 = ra::kLog2e / sqrtf((float)D);
   bp.limit_ns = wait_limit_ns();
   auto k = attn_bwd_tc_kernel<D>;
   cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_ALLOC);
-  dim3 grid(bp.nk, BH);
+  dim3 grid(bp.hgroup, bp.nk, (BH + bp.hgroup - 1) / bp.hgroup);
   Launch l(K_BWD_TC, st);
   k<<<grid, C::THREADS, C::SMEM_ALLOC, st>>>(mq, mk, mv, ml, mdq, mtab, mdk, mdv, bp);
   return RA_OK;

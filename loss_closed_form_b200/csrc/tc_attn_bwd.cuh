@@ -78,6 +78,7 @@ struct BwdParams {
   const float* lse;     // [BH][n]
   const float* delta;   // [BH][n]
   int n, BH, nk, causal;
+  int hgroup;          // heads per scheduling group (their Q~, l, dQ~ fit in L2 together)
   float scale;         // 1 / sqrt(d)
   float scale_log2;    // log2(e) / sqrt(d)
   unsigned long long limit_ns;
@@ -116,10 +117,13 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
   const uint32_t b_ep = smem_u32(&bars[12 + 2 * C::NSQ]);   // dK / dV staging written
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  // head-major order: the key tiles of one (b, h) run side by side and share its Q~, l and
-  // dQ~ in L2; key tile 0 sees the most query tiles when causal, so it goes first
-  const int kt = blockIdx.x;
-  const int bh = blockIdx.y;
+  // grid (heads of a group, key tile, group): the CTAs are dispatched x fastest, so each
+  // group of p.hgroup heads, whose Q~, l and dQ~ stay in L2 together, runs its longest key
+  // tiles first (key tile 0 sees the most query tiles when causal) across all of its heads
+  // and the grid ends on short CTAs
+  const int kt = blockIdx.y;
+  const int bh = blockIdx.z * gridDim.x + blockIdx.x;  // gridDim.x = p.hgroup
+  if (bh >= p.BH) return;  // the last group may hold fewer heads
   const int n = p.n;
   const int nqt = (n + C::BQ - 1) / C::BQ;
   const int i_start = p.causal ? (kt * C::BK) / C::BQ : 0;

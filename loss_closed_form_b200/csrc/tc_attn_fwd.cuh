@@ -70,6 +70,7 @@ struct FwdParams {
   float* delta;            // [BH][n] (with E)
   double* loss_part;       // [BH][nq][4] (with E)
   int n, BH, nq, npair, causal;
+  int hgroup;              // heads per scheduling group (their K~, V fit in L2 together)
   float scale_log2;        // log2(e) / sqrt(d)
   unsigned long long limit_ns;
 };
@@ -103,10 +104,12 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
   auto b_efull = [&](int t) { return smem_u32(&bars[8 + 4 * C::NS + t]); };  // E tile landed
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  // head-major order: the query tiles of one (b, h) run side by side and share its K~, V in
-  // L2; within a head the longest causal pairs go first
-  const int bh = blockIdx.y;
-  const int qp = p.npair - 1 - blockIdx.x;
+  // grid (heads of a group, pair rank, group): the CTAs are dispatched x fastest, so each
+  // group of p.hgroup heads, whose K~ and V stay in L2 together, runs its longest causal
+  // pairs first across all of its heads and the grid ends on short CTAs
+  const int bh = blockIdx.z * gridDim.x + blockIdx.x;  // gridDim.x = p.hgroup
+  const int qp = p.npair - 1 - blockIdx.y;
+  if (bh >= p.BH) return;  // the last group may hold fewer heads
   const int n = p.n;
   const int nk = (n + C::BN - 1) / C::BN;
   // key tiles visited by query tile t = 2 qp + t (tile 1 may lie past n: its rows are
