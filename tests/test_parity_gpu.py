@@ -189,3 +189,18 @@ def test_full_size_sampled_rows(cuda_lib, name):
     assert np.isfinite(got["loss"]) and got["loss"] > 0
     for k in ("dWQ", "dWK", "dWV"):
         assert np.all(np.isfinite(got[k]))
+
+
+@pytest.mark.slow
+def test_partial_scheduling_groups(cuda_lib):
+    """Five heads at n = 32768, d = 128: the attention kernels group heads whose re-read
+    tensors fit in 64 MB of L2 (forward 4 heads, backward 2), so the last group of each grid
+    holds fewer heads than the others and its extra CTAs leave at once.  Head 4 sits in the
+    partial group of both kernels, head 0 in a full one."""
+    w = WORKLOADS["b2_h32_n8192_d128_bf16_causal"].with_sizes(name="b1_h5_n32768_d128_bf16_causal",
+                                                             B=1, H=5, n=32768)
+    inp = make_inputs(w)
+    got = run_gpu(cuda_lib, w, inp)
+    ref = oracle.forward_backward(inp, w.causal, w.rope_base, heads=[0, 4])
+    compare(w, got, ref, heads=[0, 4])
+    _sampled_rows_check(w, inp, got, rows_per_inst=4, insts=3)
