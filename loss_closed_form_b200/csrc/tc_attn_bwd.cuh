@@ -50,7 +50,7 @@ struct BwdCfg {
   static constexpr int G_OFF = L_OFF + NSQ * QTILE;      // gamma^T, B operand of dQ~^T
   static constexpr int DQS_OFF = G_OFF + PG;              // fp32 [BQ][D] dQ~ staging tile
   static constexpr int DQS = BQ * D * 4;
-  // float [NSQ][BQ][2]: (lse * log2(e), delta) per query row
+  // float [NSQ][BQ / 2][4]: (-lse * log2(e) of rows 2i, 2i + 1, delta of rows 2i, 2i + 1)
   static constexpr int LD_OFF = DQS_OFF + DQS;
   static constexpr int BAR_OFF = LD_OFF + NSQ * BQ * 8;
   // kv_full, q_full[NSQ], q_empty[NSQ], s_full, s_free, pg_full, pg_free, dq_full, dq_free,
@@ -192,9 +192,12 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
 #pragma unroll
       for (int h = 0; h < C::BQ / 32; ++h) {
         const int c = lane + 32 * h, q = q0 + c;
-        const float lz = q < n ? p.lse[(size_t)bh * n + q] * kLog2e : 0.f;
+        const float nl = q < n ? -(p.lse[(size_t)bh * n + q] * kLog2e) : 0.f;
         const float dz = q < n ? p.delta[(size_t)bh * n + q] : 0.f;
-        st_shared_v2f(sbase + C::LD_OFF + (s * C::BQ + c) * 8, lz, dz);
+        // per column pair: (-lse_c log2 e, -lse_c+1 log2 e, delta_c, delta_c+1)
+        const uint32_t pr = sbase + C::LD_OFF + (s * C::BQ + (c & ~1)) * 8 + (c & 1) * 4;
+        st_shared_f32(pr, nl);
+        st_shared_f32(pr + 8, dz);
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(b_qfull(s));
@@ -299,19 +302,25 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       const int qh = q0 + 32 * half;
       const bool full = key < n && qh + 32 <= n && (!p.causal || key <= qh);
       uint32_t pw[16], gw[16];
+      const uint64_t sc2 = f32x2(p.scale_log2, p.scale_log2);
 #pragma unroll
       for (int h = 0; h < 16; ++h) {
         const int c = 2 * h;
-        // (lse_c, delta_c, lse_c+1, delta_c+1)
+        // (-lse_c log2 e, -lse_c+1 log2 e, delta_c, delta_c+1): two columns per packed op
         const float4 lz = ld_shared_v4f(ld_row + h * 16);
         const int q = qh + c;
         const bool v0 = full || (key < n && q < n && (!p.causal || key <= q));
         const bool v1 = full || (key < n && q + 1 < n && (!p.causal || key <= q + 1));
-        const float p0 = v0 ? ex2(__uint_as_float(sr[c]) * p.scale_log2 - lz.x) : 0.f;
-        const float p1 = v1 ? ex2(__uint_as_float(sr[c + 1]) * p.scale_log2 - lz.z) : 0.f;
+        const float2 y = unpack_f32x2(
+            ffma2(f32x2(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), sc2,
+                  f32x2(lz.x, lz.y)));
+        const float p0 = v0 ? ex2(y.x) : 0.f;
+        const float p1 = v1 ? ex2(y.y) : 0.f;
+        const float2 g = unpack_f32x2(
+            fmul2(f32x2(p0, p1), fsub2(f32x2(__uint_as_float(br[c]), __uint_as_float(br[c + 1])),
+                                       f32x2(lz.z, lz.w))));
         pw[h] = pack_bf16x2(p0, p1);
-        gw[h] = pack_bf16x2(p0 * (__uint_as_float(br[c]) - lz.y),
-                            p1 * (__uint_as_float(br[c + 1]) - lz.w));
+        gw[h] = pack_bf16x2(g.x, g.y);
       }
       // the previous tile's products have read P^T, gamma^T (TMEM) and gamma^T (smem)
       if (ii > 0) {
