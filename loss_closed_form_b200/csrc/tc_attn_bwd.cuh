@@ -308,19 +308,28 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         const int c = 2 * h;
         // (-lse_c log2 e, -lse_c+1 log2 e, delta_c, delta_c+1): two columns per packed op
         const float4 lz = ld_shared_v4f(ld_row + h * 16);
-        const int q = qh + c;
-        const bool v0 = full || (key < n && q < n && (!p.causal || key <= q));
-        const bool v1 = full || (key < n && q + 1 < n && (!p.causal || key <= q + 1));
         const float2 y = unpack_f32x2(
             ffma2(f32x2(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), sc2,
                   f32x2(lz.x, lz.y)));
-        const float p0 = v0 ? ex2(y.x) : 0.f;
-        const float p1 = v1 ? ex2(y.y) : 0.f;
+        const float p0 = ex2(y.x), p1 = ex2(y.y);
         const float2 g = unpack_f32x2(
             fmul2(f32x2(p0, p1), fsub2(f32x2(__uint_as_float(br[c]), __uint_as_float(br[c + 1])),
                                        f32x2(lz.z, lz.w))));
         pw[h] = pack_bf16x2(p0, p1);
         gw[h] = pack_bf16x2(g.x, g.y);
+      }
+      // Pairs past n or above the causal diagonal (only warps that reach the diagonal or
+      // the ragged end): their P and gamma become +0, whatever was computed there
+      if (!__all_sync(0xffffffffu, full)) {
+#pragma unroll
+        for (int h = 0; h < 16; ++h) {
+          const int q = qh + 2 * h;
+          const bool v0 = key < n && q < n && (!p.causal || key <= q);
+          const bool v1 = key < n && q + 1 < n && (!p.causal || key <= q + 1);
+          const uint32_t keep = (v0 ? 0x0000FFFFu : 0u) | (v1 ? 0xFFFF0000u : 0u);
+          pw[h] &= keep;
+          gw[h] &= keep;
+        }
       }
       // the previous tile's products have read P^T, gamma^T (TMEM) and gamma^T (smem)
       if (ii > 0) {
