@@ -9,7 +9,8 @@ tile-wise closed-form backward, inverse RoPE + weight gradients, loss reduction)
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload NAME]
 
-With N > 1 it is launched by torch.distributed.run, one process per GPU; every rank runs
+With N > 1 it runs one process per GPU under torch.distributed.run (started by the driver, or
+by bench.py itself when WORLD_SIZE is not set; a WORLD_SIZE other than N is an error); every rank runs
 its own copy of the workload (the (batch, head) instances are independent, so the work
 shards with no collective on the data path) and the reported value is the work of all
 ranks divided by the slowest rank's device time.  Rank 0 prints one JSON line.
@@ -503,8 +504,40 @@ def run_reference(args, rank, world):
                     "d2h_bytes_per_step": 0}}
 
 
+def _free_port():
+    import socket
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def launch_plan(gpus: int, env, argv, port=None):
+    """How to run `bench.py --gpus gpus`: None when this process is already the right rank
+    (one GPU, or started by torch.distributed.run with a matching world size), else the
+    torch.distributed.run command that starts one rank per GPU on this node.  A world size
+    that disagrees with --gpus is an error, not something to run."""
+    if gpus < 1:
+        raise ValueError(f"--gpus must be >= 1, got {gpus}")
+    if "WORLD_SIZE" in env:
+        world = int(env["WORLD_SIZE"])
+        if world != gpus:
+            raise ValueError(f"launched with WORLD_SIZE={world} but --gpus {gpus}")
+        return None
+    if gpus == 1:
+        return None
+    return [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+            f"--nproc-per-node={gpus}", "--master-addr=127.0.0.1",
+            f"--master-port={port if port is not None else _free_port()}",
+            os.path.join(ROOT, "bench.py"), *argv]
+
+
 def main():
     args = parse()
+    cmd = launch_plan(args.gpus, os.environ, sys.argv[1:])
+    if cmd is not None:
+        # one rank per GPU: the ranks print the JSON line (rank 0) and this process relays
+        # their exit status
+        sys.exit(subprocess.run(cmd, cwd=ROOT).returncode)
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))

@@ -60,7 +60,8 @@ typedef enum {
 
 /* One problem: B x H independent instances of n tokens with head dimension d. */
 typedef struct {
-  int32_t B, H, n, d;      /* B, H, n >= 1; d in {64, 128}                                */
+  int32_t B, H, n, d;      /* B, H, n >= 1; d in {64, 128}; B*H <= 65535; n <= 2^24, and  */
+                           /* n <= 65535*128 with bf16 I/O (else RA_ERR_UNSUPPORTED)       */
   int32_t dtype;           /* ra_dtype: element type of A1, A2, A3, E, WQ, WK, WV and O   */
   int32_t causal;          /* 0 or 1: mask keys j > i (by index)                          */
   double rope_base;        /* RoPE base, > 0 (10000, 500000, ...)                         */
@@ -87,8 +88,10 @@ size_t rope_attn_workspace_bytes(const ra_problem* p);
  *   loss : device fp32 scalar, 1/2 ||O - E||_F^2 over all instances (written); must be NULL
  *          when p->E is NULL
  *   ws   : device workspace of at least rope_attn_workspace_bytes(p) bytes
- * When p->E is given, the workspace also keeps Q~, K~, V, l and <l_i, O_i> for a following
- * rope_attn_loss_bwd(..., ws_holds_fwd = 1).
+ * When p->E is given, the workspace also keeps Q~, K~, V, l and <l_i, O_i> (and a zeroed
+ * accumulator for dQ~) for a following rope_attn_loss_bwd(..., ws_holds_fwd = 1), and its
+ * header records the problem's tag (below); without p->E the header is marked as holding
+ * nothing a backward could reuse.
  */
 ra_status rope_attn_fwd(const ra_problem* p, void* O, float* lse, float* loss,
                         void* ws, size_t ws_bytes, void* stream);
@@ -98,9 +101,18 @@ ra_status rope_attn_fwd(const ra_problem* p, void* O, float* lse, float* loss,
  *   O, lse       : device, as written by rope_attn_fwd for the same problem (read)
  *   loss         : device fp32 scalar (written; may be NULL)
  *   dWQ/dWK/dWV  : device [H][d][d] fp32 (overwritten), summed over the batch
- *   ws_holds_fwd : 1 if `ws` is the workspace of the immediately preceding rope_attn_fwd on
- *                  the same problem and inputs (with E): the projections and l are reused
- *                  instead of recomputed.  0 recomputes everything from the inputs.
+ *   ws_holds_fwd : 1 lets the device decide whether the intermediates in `ws` can be reused.
+ *                  Every forward (with E) and backward call ends by writing a header at the
+ *                  start of the workspace: a tag of the problem (B, H, n, d, dtype, causal,
+ *                  rope_base and the pos, A1, A2, A3, WQ, WK, WV, E pointers) and what the
+ *                  workspace holds.  With ws_holds_fwd = 1 the backward's recomputation
+ *                  kernels (RoPE table, projections, l = O - E and delta from the given O)
+ *                  read that header on the device and skip their work only when it carries
+ *                  this problem's tag; a workspace of another problem, of a forward without E,
+ *                  or never written is recomputed, so the result is right either way.  The
+ *                  tag sees pointers, not contents: after changing inputs in place, run
+ *                  rope_attn_fwd again (or pass 0) before the backward.
+ *                  0 recomputes everything from the inputs unconditionally.
  * p->E must not be NULL.
  */
 ra_status rope_attn_loss_bwd(const ra_problem* p, const void* O, const float* lse,
@@ -196,7 +208,9 @@ const char* rope_attn_kernel_name(int32_t id);
  *     rejected with RA_ERR_WORKSPACE before anything is launched;
  *   - the first call on a device looks up the scratch array's device address
  *     (cudaGetSymbolAddress) with that device current; make that first call before any stream
- *     capture;
+ *     capture.  Later calls reuse the address while the device's CUDA context stays the same;
+ *     after a cudaDeviceReset the next call looks it up again (so make it outside a capture
+ *     too);
  *   - every call on a device shares the one scratch array, which keeps the last call's contents;
  *     the step clears what must start at zero itself, but calls whose work overlaps on the GPU
  *     (different streams, or different host threads) race on the scratch: order them.

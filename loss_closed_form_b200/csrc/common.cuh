@@ -30,6 +30,33 @@ enum DeviceStatus : int {
 
 __device__ __forceinline__ void flag_error(int code) { atomicMax(&g_status, code); }
 
+// Header at the start of every workspace: which problem's intermediates the workspace holds.
+// The last kernel of a forward or backward call writes it; the backward's recomputation kernels
+// read it on the device and skip their work when it already holds what they would write.
+struct WsHeader {
+  unsigned long long tag;  // tag of the problem (sizes, flags, RoPE base, input pointers)
+  unsigned int magic;      // kWsMagic once written by the library
+  unsigned int state;      // kWsValid | kWsDqZero
+};
+constexpr unsigned int kWsMagic = 0x53574152u;
+constexpr unsigned int kWsValid = 1u;   // RoPE table, Q~, K~, V, l, delta and loss partials
+constexpr unsigned int kWsDqZero = 2u;  // the dQ~ accumulator holds zeros
+
+// A kernel given a gate skips its work when hdr holds `tag` with every bit of `need` set;
+// with hdr == nullptr it always works.
+struct WsGate {
+  const WsHeader* hdr;
+  unsigned long long tag;
+  unsigned int need;
+};
+
+__device__ __forceinline__ bool gate_skip(const WsGate& g) {
+  if (!g.hdr) return false;
+  const unsigned long long tag = g.hdr->tag;
+  const unsigned int magic = g.hdr->magic, state = g.hdr->state;
+  return magic == kWsMagic && tag == g.tag && (state & g.need) == g.need;
+}
+
 // Row-major [rows][cols] float tile loader with a padded smem stride.
 // Rows at or beyond `valid_rows` are filled with zeros.
 template <class T>

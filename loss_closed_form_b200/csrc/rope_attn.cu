@@ -44,13 +44,16 @@ enum KernelId : int {
   K_DA_SIMT,
   K_COMB_W,
   K_COMB_G,
+  K_PROJ_SIMT_BWD,  // launches made by a backward call (skipped on the device when the
+  K_PROJ_TC_BWD,    // workspace holds this problem's intermediates)
   K_COUNT
 };
 const char* const kKernelNames[K_COUNT] = {
-    "rope_table", "proj_rope_simt", "attn_fwd_simt", "bwd_pre",
+    "rope_table", "proj_rope_simt", "attn_fwd_simt", "bwd_prep",
     "attn_bwd_simt", "dw_partial_simt", "dw_reduce", "loss_finalize",
     "attn_fwd_tc", "attn_bwd_tc", "proj_rope_tc", "dq_unrotate", "dw_tc",
-    "input_grads_tc", "input_grads_simt", "combined_weights", "combined_grad"};
+    "input_grads_tc", "input_grads_simt", "combined_weights", "combined_grad",
+    "proj_rope_simt_bwd", "proj_rope_tc_bwd"};
 
 struct ProfRecord {
   int id;
@@ -104,6 +107,7 @@ size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 // Workspace layout.  Offsets are bytes from the workspace base, each 256-byte aligned.
 struct Layout {
+  size_t hdr;        // ra::WsHeader: which problem's intermediates the workspace holds
   size_t rope;       // float2 [n][d/2]
   size_t qt, kt, v;  // intermediate [B][H][n][d] (element size `inter`)
   size_t ell;        // intermediate [B][H][n][d]
@@ -138,11 +142,37 @@ ra_status check_problem(const ra_problem* p) {
   // grid limits: B*H blocks in y, and sizes held in 32-bit ints inside the kernels
   if ((int64_t)p->B * p->H > 65535) return RA_ERR_UNSUPPORTED;
   if ((int64_t)p->n > (1 << 24)) return RA_ERR_UNSUPPORTED;
+  // the tensor-core backward takes one CTA per 128-key tile in grid y (at most 65535)
+  if (p->dtype == RA_BF16 && (int64_t)p->n > 65535LL * 128) return RA_ERR_UNSUPPORTED;
   const void* ptrs[] = {p->A1, p->A2, p->A3, p->WQ, p->WK, p->WV, p->E};
   for (const void* q : ptrs)
     if (q && !is_aligned(q, 16)) return RA_ERR_ALIGNMENT;
   if (p->pos && !is_aligned(p->pos, 4)) return RA_ERR_ALIGNMENT;
   return RA_OK;
+}
+
+// Tag of a problem: FNV-1a over its sizes, flags, RoPE base and input pointers.  The forward
+// stamps it into the workspace header; the backward compares it on the device.
+unsigned long long problem_tag(const ra_problem* p) {
+  unsigned long long h = 1469598103934665603ull;
+  auto mix = [&](unsigned long long v) {
+    for (int i = 0; i < 8; ++i) {
+      h ^= (v >> (8 * i)) & 0xFFu;
+      h *= 1099511628211ull;
+    }
+  };
+  mix((unsigned long long)(uint32_t)p->B);
+  mix((unsigned long long)(uint32_t)p->H);
+  mix((unsigned long long)(uint32_t)p->n);
+  mix((unsigned long long)(uint32_t)p->d);
+  mix((unsigned long long)(uint32_t)p->dtype);
+  mix((unsigned long long)(uint32_t)p->causal);
+  unsigned long long base_bits;
+  memcpy(&base_bits, &p->rope_base, sizeof(base_bits));
+  mix(base_bits);
+  const void* ptrs[] = {p->pos, p->A1, p->A2, p->A3, p->WQ, p->WK, p->WV, p->E};
+  for (const void* q : ptrs) mix((unsigned long long)(uintptr_t)q);
+  return h;
 }
 
 Layout make_layout(const ra_problem* p) {
@@ -177,6 +207,7 @@ Layout make_layout(const ra_problem* p) {
     off = align_up(off + bytes, kAlignWs);
     return o;
   };
+  L.hdr = take(sizeof(ra::WsHeader));
   L.rope = take(n * (d / 2) * sizeof(float2));
   L.qt = take(act * L.inter);
   L.kt = take(act * L.inter);
@@ -306,28 +337,78 @@ bool map_f32_3d(CUtensorMap* m, void* base, uint64_t cols, uint64_t rows, uint64
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Last launch of every forward and backward call: the loss (when asked for) from the partial
+// sums, then the workspace header (this problem's tag and `state`).  `count` partials belong to
+// this call; when `gate` finds the recomputation skipped, the forward's partials are summed.
+void finalize(const ra_problem* p, const Layout& L, void* ws, float* loss, int count,
+              ra::WsGate gate, unsigned int state, cudaStream_t st) {
+  Launch l(K_LOSS, st);
+  ra::simt::loss_finalize_kernel<<<1, 1024, 0, st>>>(at<double>(ws, L.loss_part), count,
+                                                    L.nparts_fwd, loss, gate,
+                                                    at<ra::WsHeader>(ws, L.hdr), problem_tag(p),
+                                                    state);
+}
+
+// RoPE table of the forward (grid-stride, a few blocks per SM).
+void rope_table(const ra_problem* p, const Layout& L, void* ws, cudaStream_t st) {
+  const long long total = (long long)p->n * (p->d / 2);
+  const long long want = (total + 255) / 256, cap = 8LL * num_sms();
+  Launch l(K_ROPE_TABLE, st);
+  ra::simt::rope_table_kernel<<<(unsigned)(want < cap ? want : cap), 256, 0, st>>>(
+      at<float2>(ws, L.rope), p->pos, p->n, p->d / 2, p->rope_base);
+}
+
+// Gates of the backward.  With ws_holds_fwd the device decides from the workspace header:
+// the recomputation (RoPE table, projections, l and delta) is skipped when the header holds
+// this problem's intermediates, the zeroing of dQ~ when it is zero already.  Without, both run.
+struct BwdGates {
+  ra::WsGate recompute, zero;
+};
+BwdGates bwd_gates(const ra_problem* p, const Layout& L, void* ws, int holds) {
+  const ra::WsHeader* hdr = holds ? at<ra::WsHeader>(ws, L.hdr) : nullptr;
+  const unsigned long long tag = problem_tag(p);
+  return BwdGates{ra::WsGate{hdr, tag, ra::kWsValid},
+                  ra::WsGate{hdr, tag, ra::kWsValid | ra::kWsDqZero}};
+}
+
+// The backward's preparation (one launch): unless the gates find the workspace ready, the
+// RoPE table, l = O - E, delta and the loss partials, and the zeroing of dQ~.
+template <class T, class TL>
+void bwd_prep(const ra_problem* p, const Layout& L, const void* O, void* ws, const BwdGates& g,
+              cudaStream_t st) {
+  const long long BH = (long long)p->B * p->H;
+  const long long vblocks = BH * ((p->n + ra::simt::kRows - 1) / ra::simt::kRows);
+  const long long cap = 8LL * num_sms();
+  Launch l(K_BWD_PRE, st);
+  ra::simt::bwd_prep_kernel<T, TL><<<(unsigned)(vblocks < cap ? vblocks : cap),
+                                     ra::simt::kThreads, 0, st>>>(
+      (const T*)O, (const T*)p->E, at<TL>(ws, L.ell), at<float>(ws, L.delta),
+      at<double>(ws, L.loss_part), p->n, p->d, (int)BH, at<float2>(ws, L.rope), p->pos,
+      p->rope_base, at<float4>(ws, L.dqt), BH * p->n * p->d / 4, g.recompute, g.zero);
+}
+
 // ---------------------------------------------------------------------------------------
 // fp32 CUDA-core path
 // ---------------------------------------------------------------------------------------
+// Projections + RoPE from the table in the workspace.  The gate (hdr == nullptr: none) lets
+// the kernel skip the work on the device when the workspace already holds this problem's
+// projections.
 template <class T, class TX>
-ra_status simt_project(const ra_problem* p, const Layout& L, void* ws, cudaStream_t st) {
+ra_status simt_project(const ra_problem* p, const Layout& L, void* ws, ra::WsGate gate,
+                       bool in_bwd, cudaStream_t st) {
   using namespace ra::simt;
-  const int n = p->n, d = p->d, half = d / 2;
+  const int n = p->n, d = p->d;
   float2* tab = at<float2>(ws, L.rope);
-  {
-    int total = n * half;
-    Launch l(K_ROPE_TABLE, st);
-    rope_table_kernel<<<(total + 255) / 256, 256, 0, st>>>(tab, p->pos, n, half, p->rope_base);
-  }
   {
     size_t smem = (size_t)(kRows * (d + 4) + d * d) * sizeof(float);
     auto k = proj_rope_kernel<T, TX>;
     cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     dim3 grid((n + kRows - 1) / kRows, p->B * p->H, 3);
-    Launch l(K_PROJ_SIMT, st);
+    Launch l(in_bwd ? K_PROJ_SIMT_BWD : K_PROJ_SIMT, st);
     k<<<grid, kThreads, smem, st>>>(
         (const T*)p->A1, (const T*)p->A2, (const T*)p->A3, (const T*)p->WQ, (const T*)p->WK,
-        (const T*)p->WV, tab, at<TX>(ws, L.qt), at<TX>(ws, L.kt), at<TX>(ws, L.v), p->H, n, d);
+        (const T*)p->WV, tab, at<TX>(ws, L.qt), at<TX>(ws, L.kt), at<TX>(ws, L.v), p->H, n, d,
+        gate);
   }
   return launch_status();
 }
@@ -337,7 +418,8 @@ ra_status simt_fwd(const ra_problem* p, void* O, float* lse, float* loss, void* 
                    cudaStream_t st) {
   using namespace ra::simt;
   const Layout L = make_layout(p);
-  ra_status s = simt_project<T, float>(p, L, ws, st);
+  rope_table(p, L, ws, st);
+  ra_status s = simt_project<T, float>(p, L, ws, ra::WsGate{nullptr, 0, 0}, false, st);
   if (s != RA_OK) return s;
   const int n = p->n, d = p->d;
   const float scale = 1.0f / sqrtf((float)d);
@@ -352,10 +434,8 @@ ra_status simt_fwd(const ra_problem* p, void* O, float* lse, float* loss, void* 
                                     at<float>(ws, L.delta), at<double>(ws, L.loss_part), n, d,
                                     p->causal, scale * ra::kLog2e);
   }
-  if (loss) {
-    Launch l(K_LOSS, st);
-    loss_finalize_kernel<<<1, 1024, 0, st>>>(at<double>(ws, L.loss_part), L.nparts_fwd, loss);
-  }
+  // loss, then the header: with a target the workspace now holds l, delta and the partials
+  finalize(p, L, ws, loss, L.nparts_fwd, ra::WsGate{nullptr, 0, 0}, p->E ? ra::kWsValid : 0u, st);
   return launch_status();
 }
 
@@ -363,17 +443,12 @@ ra_status simt_fwd(const ra_problem* p, void* O, float* lse, float* loss, void* 
 // bf16 tensor-core path
 // ---------------------------------------------------------------------------------------
 template <int D>
-ra_status tc_project(const ra_problem* p, const Layout& L, void* ws, cudaStream_t st) {
+ra_status tc_project(const ra_problem* p, const Layout& L, void* ws, ra::WsGate gate,
+                     bool in_bwd, cudaStream_t st) {
   using namespace ra::tc;
   using C = ProjCfg<D>;
-  const int n = p->n, BH = p->B * p->H, half = D / 2;
+  const int n = p->n, BH = p->B * p->H;
   float2* tab = at<float2>(ws, L.rope);
-  {
-    int total = n * half;
-    Launch l(K_ROPE_TABLE, st);
-    ra::simt::rope_table_kernel<<<(total + 255) / 256, 256, 0, st>>>(tab, p->pos, n, half,
-                                                                     p->rope_base);
-  }
   CUtensorMap a1, a2, a3, w1, w2, w3, o1, o2, o3;
   if (!map_bf16_3d(&a1, p->A1, D, n, BH, C::BM) || !map_bf16_3d(&a2, p->A2, D, n, BH, C::BM) ||
       !map_bf16_3d(&a3, p->A3, D, n, BH, C::BM) || !map_bf16_3d(&w1, p->WQ, D, D, p->H, D) ||
@@ -395,9 +470,10 @@ ra_status tc_project(const ra_problem* p, const Layout& L, void* ws, cudaStream_
   pp.tiles_per_cta = (pp.tiles + ctas - 1) / ctas;
   const long long grid = (pp.tiles + pp.tiles_per_cta - 1) / pp.tiles_per_cta;
   pp.limit_ns = wait_limit_ns();
+  pp.gate = gate;
   auto k = proj_rope_tc_kernel<D, false>;
   cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_ALLOC);
-  Launch l(K_PROJ_TC, st);
+  Launch l(in_bwd ? K_PROJ_TC_BWD : K_PROJ_TC, st);
   k<<<(unsigned)grid, C::THREADS, C::SMEM_ALLOC, st>>>(a1, a2, a3, w1, w2, w3, o1, o2, o3, pp);
   return launch_status();
 }
@@ -430,6 +506,7 @@ ra_status tc_input_grads(const ra_problem* p, const Layout& L, void* dA1, void* 
   pp.tiles_per_cta = (pp.tiles + ctas - 1) / ctas;
   const long long grid = (pp.tiles + pp.tiles_per_cta - 1) / pp.tiles_per_cta;
   pp.limit_ns = wait_limit_ns();
+  pp.gate = ra::WsGate{nullptr, 0, 0};
   auto k = proj_rope_tc_kernel<D, true>;
   cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_ALLOC);
   Launch l(K_DA_TC, st);
@@ -457,7 +534,7 @@ ra_status simt_input_grads(const ra_problem* p, const Layout& L, void* dA1, void
 
 template <int D>
 ra_status tc_weight_grads(const ra_problem* p, const Layout& L, float* dWQ, float* dWK,
-                          float* dWV, void* ws, cudaStream_t st) {
+                          float* dWV, void* ws, ra::WsHeader* stamp, cudaStream_t st) {
   using namespace ra::tc;
   using C = DwCfg<D>;
   const int n = p->n, BH = p->B * p->H, half = D / 2;
@@ -495,7 +572,8 @@ ra_status tc_weight_grads(const ra_problem* p, const Layout& L, float* dWQ, floa
     size_t total = (size_t)3 * p->H * D * D;
     Launch l(K_DW_REDUCE, st);
     ra::simt::dw_reduce_kernel<<<(unsigned)((total + 255) / 256), 256, 0, st>>>(
-        at<float>(ws, L.dw_part), dWQ, dWK, dWV, p->H, D, L.nsplit);
+        at<float>(ws, L.dw_part), dWQ, dWK, dWV, p->H, D, L.nsplit, stamp, problem_tag(p),
+        ra::kWsValid);
   }
   return launch_status();
 }
@@ -521,6 +599,8 @@ ra_status tc_fwd_launch(const ra_problem* p, const Layout& L, void* O, float* ls
   fp.ell = at<__nv_bfloat16>(ws, L.ell);
   fp.delta = at<float>(ws, L.delta);
   fp.loss_part = at<double>(ws, L.loss_part);
+  // with a target the backward will follow: zero its dQ~ accumulator on the forward's idle warps
+  fp.dq_zero = p->E ? at<float>(ws, L.dqt) : nullptr;
   fp.n = n;
   fp.BH = BH;
   fp.nq = (n + C::BM - 1) / C::BM;
@@ -540,16 +620,15 @@ ra_status tc_fwd_launch(const ra_problem* p, const Layout& L, void* O, float* ls
 ra_status tc_fwd(const ra_problem* p, void* O, float* lse, float* loss, void* ws,
                  cudaStream_t st) {
   const Layout L = make_layout(p);
-  ra_status s = p->d == 128 ? tc_project<128>(p, L, ws, st) : tc_project<64>(p, L, ws, st);
+  const ra::WsGate none{nullptr, 0, 0};
+  rope_table(p, L, ws, st);
+  ra_status s = p->d == 128 ? tc_project<128>(p, L, ws, none, false, st)
+                            : tc_project<64>(p, L, ws, none, false, st);
   if (s != RA_OK) return s;
   s = p->d == 128 ? tc_fwd_launch<128>(p, L, O, lse, ws, st)
                   : tc_fwd_launch<64>(p, L, O, lse, ws, st);
   if (s != RA_OK) return s;
-  if (loss) {
-    Launch l(K_LOSS, st);
-    ra::simt::loss_finalize_kernel<<<1, 1024, 0, st>>>(at<double>(ws, L.loss_part), L.nparts_fwd,
-                                                      loss);
-  }
+  finalize(p, L, ws, loss, L.nparts_fwd, none, p->E ? (ra::kWsValid | ra::kWsDqZero) : 0u, st);
   return launch_status();
 }
 
@@ -594,18 +673,12 @@ ra_status simt_bwd(const ra_problem* p, const void* O, const float* lse, float* 
   using namespace ra::simt;
   const Layout L = make_layout(p);
   const int n = p->n, d = p->d;
-  if (!holds) {
-    ra_status s = simt_project<float, float>(p, L, ws, st);
+  const BwdGates g = bwd_gates(p, L, ws, holds);
+  bwd_prep<float, float>(p, L, O, ws, g, st);
+  {
+    ra_status s = simt_project<float, float>(p, L, ws, g.recompute, true, st);
     if (s != RA_OK) return s;
-    dim3 grid((n + kRows - 1) / kRows, p->B * p->H);
-    Launch l(K_BWD_PRE, st);
-    bwd_pre_kernel<float, float><<<grid, kThreads, 0, st>>>(
-        (const float*)O, (const float*)p->E, at<float>(ws, L.ell), at<float>(ws, L.delta),
-        at<double>(ws, L.loss_part), n, d);
   }
-  const size_t act = (size_t)p->B * p->H * n * d;
-  if (cudaMemsetAsync(at<float>(ws, L.dqt), 0, act * sizeof(float), st) != cudaSuccess)
-    return RA_ERR_CUDA;
   const float scale = 1.0f / sqrtf((float)d);
   {
     size_t smem = (size_t)(4 * kRows * (d + 4) + 2 * kRows * 33 + 2 * kRows) * sizeof(float);
@@ -630,14 +703,13 @@ ra_status simt_bwd(const ra_problem* p, const void* O, const float* lse, float* 
     }
     size_t total = (size_t)3 * p->H * d * d;
     Launch l(K_DW_REDUCE, st);
+    // the workspace now holds this problem's intermediates and dQ~ is no longer zero: the
+    // header says so, written by the last launch of the call
     dw_reduce_kernel<<<(unsigned)((total + 255) / 256), 256, 0, st>>>(
-        at<float>(ws, L.dw_part), dWQ, dWK, dWV, p->H, d, L.nsplit);
+        at<float>(ws, L.dw_part), dWQ, dWK, dWV, p->H, d, L.nsplit,
+        loss ? nullptr : at<ra::WsHeader>(ws, L.hdr), problem_tag(p), ra::kWsValid);
   }
-  if (loss) {
-    Launch l(K_LOSS, st);
-    loss_finalize_kernel<<<1, 1024, 0, st>>>(at<double>(ws, L.loss_part),
-                                            holds ? L.nparts_fwd : L.nparts_pre, loss);
-  }
+  if (loss) finalize(p, L, ws, loss, L.nparts_pre, g.recompute, ra::kWsValid, st);
   return launch_status();
 }
 
@@ -645,30 +717,21 @@ ra_status simt_bwd(const ra_problem* p, const void* O, const float* lse, float* 
 ra_status tc_bwd(const ra_problem* p, const void* O, const float* lse, float* loss, float* dWQ,
                  float* dWK, float* dWV, void* ws, int holds, cudaStream_t st) {
   const Layout L = make_layout(p);
-  const int n = p->n, d = p->d;
-  ra_status s;
-  if (!holds) {
-    s = d == 128 ? tc_project<128>(p, L, ws, st) : tc_project<64>(p, L, ws, st);
-    if (s != RA_OK) return s;
-    dim3 grid((n + ra::simt::kRows - 1) / ra::simt::kRows, p->B * p->H);
-    Launch l(K_BWD_PRE, st);
-    ra::simt::bwd_pre_kernel<__nv_bfloat16, __nv_bfloat16><<<grid, ra::simt::kThreads, 0, st>>>(
-        (const __nv_bfloat16*)O, (const __nv_bfloat16*)p->E, at<__nv_bfloat16>(ws, L.ell),
-        at<float>(ws, L.delta), at<double>(ws, L.loss_part), n, d);
-  }
-  const size_t act = (size_t)p->B * p->H * n * d;
-  if (cudaMemsetAsync(at<float>(ws, L.dqt), 0, act * sizeof(float), st) != cudaSuccess)
-    return RA_ERR_CUDA;
+  const int d = p->d;
+  const BwdGates g = bwd_gates(p, L, ws, holds);
+  bwd_prep<__nv_bfloat16, __nv_bfloat16>(p, L, O, ws, g, st);
+  ra_status s = d == 128 ? tc_project<128>(p, L, ws, g.recompute, true, st)
+                         : tc_project<64>(p, L, ws, g.recompute, true, st);
+  if (s != RA_OK) return s;
   s = d == 128 ? tc_bwd_launch<128>(p, L, lse, ws, st) : tc_bwd_launch<64>(p, L, lse, ws, st);
   if (s != RA_OK) return s;
-  s = d == 128 ? tc_weight_grads<128>(p, L, dWQ, dWK, dWV, ws, st)
-               : tc_weight_grads<64>(p, L, dWQ, dWK, dWV, ws, st);
+  // the workspace now holds this problem's intermediates and dQ~ is no longer zero: the header
+  // says so, written by the last launch of the call (loss_finalize when there is a loss to sum)
+  ra::WsHeader* stamp = loss ? nullptr : at<ra::WsHeader>(ws, L.hdr);
+  s = d == 128 ? tc_weight_grads<128>(p, L, dWQ, dWK, dWV, ws, stamp, st)
+               : tc_weight_grads<64>(p, L, dWQ, dWK, dWV, ws, stamp, st);
   if (s != RA_OK) return s;
-  if (loss) {
-    Launch l(K_LOSS, st);
-    ra::simt::loss_finalize_kernel<<<1, 1024, 0, st>>>(at<double>(ws, L.loss_part),
-                                                      holds ? L.nparts_fwd : L.nparts_pre, loss);
-  }
+  if (loss) finalize(p, L, ws, loss, L.nparts_pre, g.recompute, ra::kWsValid, st);
   return launch_status();
 }
 
@@ -682,17 +745,52 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[RA_NOALLOC_SCRA
 constexpr int kMaxDevices = 64;
 std::mutex g_noalloc_mutex;
 void* g_noalloc_addr[kMaxDevices] = {};
+unsigned long long g_noalloc_ctx[kMaxDevices] = {};
 
-// Device address of the scratch array on the current device (looked up once per device).
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+
+// Unique id of the calling thread's current CUDA context, 0 if there is none or the driver
+// cannot tell.  A device reset destroys the context that held the scratch array; the context
+// created after it has a new id, and the array may sit at a new address there.
+unsigned long long current_ctx_id() {
+  static CtxGetCurrentFn get_cur = [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    return (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) ==
+                cudaSuccess && q == cudaDriverEntryPointSuccess)
+               ? reinterpret_cast<CtxGetCurrentFn>(f)
+               : (CtxGetCurrentFn) nullptr;
+  }();
+  static CtxGetIdFn get_id = [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    return (cudaGetDriverEntryPoint("cuCtxGetId", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+               ? reinterpret_cast<CtxGetIdFn>(f)
+               : (CtxGetIdFn) nullptr;
+  }();
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (!get_cur || !get_id || get_cur(&ctx) != CUDA_SUCCESS || !ctx) return 0;
+  if (get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
+
+// Device address of the scratch array on the current device: looked up with the device
+// current on its first use, and again whenever the device's context has changed since (after a
+// device reset) or cannot be identified.
 ra_status noalloc_scratch(void** out) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess) return RA_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDevices) return RA_ERR_UNSUPPORTED;
   std::lock_guard<std::mutex> lock(g_noalloc_mutex);
-  if (!g_noalloc_addr[dev]) {
+  const unsigned long long id = current_ctx_id();
+  if (!g_noalloc_addr[dev] || id == 0 || id != g_noalloc_ctx[dev]) {
     void* ptr = nullptr;
     if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr) return RA_ERR_CUDA;
     g_noalloc_addr[dev] = ptr;
+    g_noalloc_ctx[dev] = current_ctx_id();  // the lookup made the primary context current
   }
   *out = g_noalloc_addr[dev];
   return RA_OK;

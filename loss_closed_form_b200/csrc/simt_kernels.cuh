@@ -15,17 +15,32 @@ constexpr int kThreads = 256;  // 8 threads per row
 
 // ---------------------------------------------------------------------------------------
 // RoPE table: tab[i][k] = (cos, sin)(pos_i * base^(-2k/d)), angle and sin/cos in fp64.
+// Grid-stride over the n * half entries; each block first puts theta_k = base^(-2k/d) for the
+// half <= 64 frequencies in shared memory, so pow runs once per block and frequency.
 // ---------------------------------------------------------------------------------------
+constexpr int kMaxHalf = 64;
+
+__device__ __forceinline__ void rope_table_fill(float2* __restrict__ tab,
+                                                const int32_t* __restrict__ pos, int n, int half,
+                                                double base) {
+  __shared__ double theta[kMaxHalf];
+  for (int k = threadIdx.x; k < half; k += blockDim.x)
+    theta[k] = pow(base, -2.0 * (double)k / (double)(2 * half));
+  __syncthreads();
+  const long long total = (long long)n * half;
+  for (long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
+       idx += (long long)gridDim.x * blockDim.x) {
+    const int i = (int)(idx / half), k = (int)(idx - (long long)i * half);
+    const double p = pos ? (double)pos[i] : (double)i;
+    double sn, cs;
+    sincos(p * theta[k], &sn, &cs);
+    tab[idx] = make_float2((float)cs, (float)sn);
+  }
+}
+
 __global__ void rope_table_kernel(float2* __restrict__ tab, const int32_t* __restrict__ pos,
                                   int n, int half, double base) {
-  int idx = blockIdx.x * blockDim.x + threadIdx.x;
-  if (idx >= n * half) return;
-  int i = idx / half, k = idx - i * half;
-  double p = pos ? (double)pos[i] : (double)i;
-  double theta = pow(base, -2.0 * (double)k / (double)(2 * half));
-  double s, c;
-  sincos(p * theta, &s, &c);
-  tab[idx] = make_float2((float)c, (float)s);
+  rope_table_fill(tab, pos, n, half, base);
 }
 
 // ---------------------------------------------------------------------------------------
@@ -37,7 +52,8 @@ __global__ void __launch_bounds__(kThreads)
 proj_rope_kernel(const TI* __restrict__ A1, const TI* __restrict__ A2, const TI* __restrict__ A3,
                  const TI* __restrict__ WQ, const TI* __restrict__ WK, const TI* __restrict__ WV,
                  const float2* __restrict__ tab, TO* __restrict__ Qt, TO* __restrict__ Kt,
-                 TO* __restrict__ Vo, int H, int n, int d) {
+                 TO* __restrict__ Vo, int H, int n, int d, WsGate gate) {
+  if (gate_skip(gate)) return;
   extern __shared__ float smem[];
   const int ld = d + 4;
   float* As = smem;             // [32][d+4]
@@ -196,24 +212,26 @@ attn_fwd_kernel(const float* __restrict__ Qt, const float* __restrict__ Kt,
 }
 
 // ---------------------------------------------------------------------------------------
-// l = O - E, delta_i = <l_i, O_i>, partial sums of 1/2 l^2, from a given O (I/O dtype).
-// grid (ceil(n/32), B*H), 256 threads.
+// l = O - E, delta_i = <l_i, O_i>, partial sums of 1/2 l^2, from a given O (I/O dtype), for
+// the 32 rows of row block rb of instance bh (256 threads, 8 per row); the block's partial sum
+// goes to loss_part[bh * nrb + rb].
 // ---------------------------------------------------------------------------------------
 template <class T, class TL>
-__global__ void __launch_bounds__(kThreads)
-bwd_pre_kernel(const T* __restrict__ O, const T* __restrict__ E, TL* __restrict__ ell,
-               float* __restrict__ delta, double* __restrict__ loss_part, int n, int d) {
-  __shared__ double red[kThreads / 32];
-  const int bh = blockIdx.y, tid = threadIdx.x, r = tid >> 3, g = tid & 7;
-  const int row = blockIdx.x * kRows + r;
+__device__ __forceinline__ void bwd_pre_rows(const T* __restrict__ O, const T* __restrict__ E,
+                                             TL* __restrict__ ell, float* __restrict__ delta,
+                                             double* __restrict__ loss_part, int n, int d,
+                                             int bh, int rb, int nrb, double* red) {
+  const int tid = threadIdx.x, r = tid >> 3, g = tid & 7;
+  const int row = rb * kRows + r;
   float dl = 0.f, sq = 0.f;
   if (row < n) {
     const size_t ro = ((size_t)bh * n + row) * d;
     for (int col = g; col < d; col += 8) {
       float o = to_f(O[ro + col]);
       float e = o - to_f(E[ro + col]);
-      ell[ro + col] = from_f<TL>(e);
-      dl = fmaf(e, o, dl);
+      const TL er = from_f<TL>(e);
+      ell[ro + col] = er;
+      dl = fmaf(to_f(er), o, dl);  // delta from the stored l, which beta is built from
       sq = fmaf(e, e, sq);
     }
   }
@@ -231,8 +249,37 @@ bwd_pre_kernel(const T* __restrict__ O, const T* __restrict__ E, TL* __restrict_
   if (tid == 0) {
     double t = 0.0;
     for (int w = 0; w < kThreads / 32; ++w) t += red[w];
-    loss_part[(size_t)blockIdx.y * gridDim.x + blockIdx.x] = t;
+    loss_part[(size_t)bh * nrb + rb] = t;
   }
+  __syncthreads();  // red is reused by the block's next row block
+}
+
+// The backward's preparation in one launch (grid-stride, 256 threads per block):
+//   unless `recompute` is skipped: the RoPE table and, for every 32-row block of every
+//     instance, l = O - E, delta and the loss partial (nrb row blocks per instance);
+//   unless `zero` is skipped: the dQ~ accumulator (n4 float4) is set to zero.
+// Both gates read the workspace header; when it holds this problem's intermediates and a
+// zeroed accumulator, the whole launch returns at once.
+template <class T, class TL>
+__global__ void __launch_bounds__(kThreads)
+bwd_prep_kernel(const T* __restrict__ O, const T* __restrict__ E, TL* __restrict__ ell,
+                float* __restrict__ delta, double* __restrict__ loss_part, int n, int d, int BH,
+                float2* __restrict__ tab, const int32_t* __restrict__ pos, double base,
+                float4* __restrict__ dq, long long n4, WsGate recompute, WsGate zero) {
+  __shared__ double red[kThreads / 32];
+  const bool rec = !gate_skip(recompute), zer = !gate_skip(zero);
+  if (rec) {
+    rope_table_fill(tab, pos, n, d / 2, base);
+    const int nrb = (n + kRows - 1) / kRows;
+    const long long nvb = (long long)nrb * BH;
+    for (long long vb = blockIdx.x; vb < nvb; vb += gridDim.x)
+      bwd_pre_rows<T, TL>(O, E, ell, delta, loss_part, n, d, (int)(vb / nrb), (int)(vb % nrb),
+                          nrb, red);
+  }
+  if (zer)
+    for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n4;
+         i += (long long)gridDim.x * blockDim.x)
+      dq[i] = make_float4(0.f, 0.f, 0.f, 0.f);
 }
 
 // ---------------------------------------------------------------------------------------
@@ -417,11 +464,19 @@ dw_partial_kernel(const TA* __restrict__ A1, const TA* __restrict__ A2, const TA
 }
 
 // dW[z][h] = sum over splits (fixed order) of part[z][h][split].
+// When `stamp` is given (a backward without a loss to sum, so no loss_finalize follows),
+// thread 0 also writes the workspace header (stamp_tag, stamp_state).
 __global__ void dw_reduce_kernel(const float* __restrict__ part, float* __restrict__ dWQ,
                                  float* __restrict__ dWK, float* __restrict__ dWV, int H, int d,
-                                 int nsplit) {
+                                 int nsplit, WsHeader* stamp, unsigned long long stamp_tag,
+                                 unsigned int stamp_state) {
   const size_t dd = (size_t)d * d;
   const size_t idx = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (stamp && idx == 0) {
+    stamp->tag = stamp_tag;
+    stamp->state = stamp_state;
+    stamp->magic = kWsMagic;
+  }
   if (idx >= 3 * H * dd) return;
   const int z = (int)(idx / (H * dd));
   const size_t rem = idx - (size_t)z * H * dd;
@@ -434,12 +489,24 @@ __global__ void dw_reduce_kernel(const float* __restrict__ part, float* __restri
   dW[(size_t)h * dd + e] = (float)s;
 }
 
-// loss = sum of the partials in a fixed order (fp64), one block of 256 threads.
-__global__ void loss_finalize_kernel(const double* __restrict__ part, int count,
-                                     float* __restrict__ loss) {
+// Last kernel of a forward or backward call (one block): loss = sum of the partials in a
+// fixed order (fp64), when `loss` is given, then the workspace header is stamped with
+// (stamp_tag, stamp_state).  The partials are the `count_kept` ones an earlier forward left
+// when `gate` skipped the backward's recomputation, else the `count` ones of this call.
+__global__ void loss_finalize_kernel(const double* __restrict__ part, int count, int count_kept,
+                                     float* __restrict__ loss, WsGate gate, WsHeader* stamp,
+                                     unsigned long long stamp_tag, unsigned int stamp_state) {
   // fixed summation order for a given count and block size (deterministic); four
   // independent partial sums per thread keep the loads in flight
   __shared__ double red[1024];
+  if (gate_skip(gate)) count = count_kept;
+  __syncthreads();  // every thread has read the header before thread 0 rewrites it
+  if (stamp && threadIdx.x == 0) {
+    stamp->tag = stamp_tag;
+    stamp->state = stamp_state;
+    stamp->magic = kWsMagic;
+  }
+  if (!loss) return;
   double s0 = 0.0, s1 = 0.0, s2 = 0.0, s3 = 0.0;
   const int stride = blockDim.x;
   int i = threadIdx.x;

@@ -21,11 +21,13 @@
 // log2(e)/sqrt(d) > 0 is applied to it and folded into each exponent's FFMA.
 //
 // Warp roles (384 threads): warps 0-3 softmax + epilogue of query tile 0, warps 4-7 of
-// query tile 1, warp 8 TMA producer, warp 9 MMA issuer and TMEM owner, warps 10-11 idle.
+// query tile 1, warp 8 TMA producer, warp 9 MMA issuer and TMEM owner, warps 10-11 zero the
+// pair's rows of the backward's dQ~ accumulator (when asked to) and are otherwise idle.
 // The third warpgroup hands registers to the two softmax warpgroups (setmaxnreg): a thread
 // there holds a whole 128-column row of scores.
 #pragma once
 #include "tc_ptx.cuh"
+
 
 namespace ra {
 namespace tc {
@@ -69,6 +71,7 @@ struct FwdParams {
   __nv_bfloat16* ell;      // [BH][n][d] (with E)
   float* delta;            // [BH][n] (with E)
   double* loss_part;       // [BH][nq][4] (with E)
+  float* dq_zero;          // [BH][n][d] fp32 accumulator of the backward, zeroed here, or null
   int n, BH, nq, npair, causal;
   int hgroup;              // heads per scheduling group (their K~, V fit in L2 together)
   float scale_log2;        // log2(e) / sqrt(d)
@@ -392,11 +395,16 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
               const __nv_bfloat162 e2 = *reinterpret_cast<const __nv_bfloat162*>(&ew[q]);
               const float e0 = o[2 * q] - __low2float(e2);
               const float e1 = o[2 * q + 1] - __high2float(e2);
+              const uint32_t lr = pack_bf16x2(e0, e1);
+              lw[16 * c + 4 * v + q] = lr;
               if (vrow) {
-                dl = fmaf(e0, o[2 * q], fmaf(e1, o[2 * q + 1], dl));
+                // delta from the stored (bf16) l, the l the backward's beta = l V^T is built
+                // from: then sum_j s_ij (beta_ij - delta_i) = 0 holds for the rounded l too, and
+                // rows with one key (s = 1) get gamma = 0 exactly; the loss keeps the fp32 l
+                const __nv_bfloat162 l2 = *reinterpret_cast<const __nv_bfloat162*>(&lr);
+                dl = fmaf(__low2float(l2), o[2 * q], fmaf(__high2float(l2), o[2 * q + 1], dl));
                 sq = fmaf(e0, e0, fmaf(e1, e1, sq));
               }
-              lw[16 * c + 4 * v + q] = pack_bf16x2(e0, e1);
             }
           }
           st_shared_v4(a, pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]),
@@ -441,6 +449,18 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
     for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
     if (p.E && ok && lane == 0 && qt < p.nq)
       p.loss_part[((size_t)bh * p.nq + qt) * C::LOSS_PARTS + (warp & 3)] = 0.5 * (double)sq;
+  } else if (p.dq_zero) {
+    // ------------------------------------------------------------------ warps 10-11
+    // zero rows 2 qp * 128 .. of this instance's dQ~ accumulator (the pair's two query tiles,
+    // clipped to n): every row of every instance belongs to exactly one pair
+    const int r0 = 2 * qp * C::BM;
+    const int r1 = min(n, r0 + 2 * C::BM);
+    if (r1 > r0) {
+      float4* dst = reinterpret_cast<float4*>(p.dq_zero + ((size_t)bh * n + r0) * D);
+      const int cnt = (r1 - r0) * (D / 4);
+      for (int i = tid - 32 * (C::W_MMA + 1); i < cnt; i += 64)
+        dst[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
   }
   tc_fence_before();
   __syncthreads();

@@ -58,6 +58,7 @@ struct ProjParams {
   long long tiles;         // B * nrt * 3 * H
   long long tiles_per_cta;
   unsigned long long limit_ns;
+  WsGate gate;             // skip everything when the workspace already holds the outputs
 };
 
 template <int D, bool IG>
@@ -68,6 +69,7 @@ proj_rope_tc_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_cons
                     const __grid_constant__ CUtensorMap tm_o1, const __grid_constant__ CUtensorMap tm_o2,
                     const __grid_constant__ CUtensorMap tm_o3, const ProjParams p) {
   using C = ProjCfg<D>;
+  if (gate_skip(p.gate)) return;  // uniform over the grid, before any barrier or TMEM use
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));

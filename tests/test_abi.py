@@ -77,6 +77,10 @@ def test_workspace_bytes():
     (dict(WV=None), ra.RA_ERR_INVALID_ARG),
     (dict(d=32), ra.RA_ERR_UNSUPPORTED),
     (dict(d=256), ra.RA_ERR_UNSUPPORTED),
+    # bf16: the backward's grid holds one CTA per 128-key tile in y (at most 65535)
+    (dict(n=65535 * 128 + 1, dtype=ra.RA_BF16), ra.RA_ERR_UNSUPPORTED),
+    (dict(n=(1 << 24) + 1, dtype=ra.RA_F32), ra.RA_ERR_UNSUPPORTED),
+    (dict(B=300, H=300), ra.RA_ERR_UNSUPPORTED),
     (dict(A2=FAKE + 8), ra.RA_ERR_ALIGNMENT),
     (dict(E=FAKE + 2), ra.RA_ERR_ALIGNMENT),
     (dict(pos=FAKE + 2), ra.RA_ERR_ALIGNMENT),

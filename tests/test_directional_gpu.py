@@ -3,7 +3,9 @@ these sizes):
 
   * the directional derivative of the loss along a random direction P of (WQ, WK, WV), by
     central differences of the GPU forward, (L(W + eps P) - L(W - eps P)) / (2 eps), against
-    <grad L, P> from the GPU backward (fp32 path, B=2 H=32 n=8192 d=128 causal).  The central
+    <grad L, P> from the GPU backward (fp32 path) at the three long-sequence workloads:
+    B=2 H=32 n=8192, B=1 H=8 n=32768 with bounded scores, and B=1 H=8 n=131072 with RoPE
+    base 5e5 (d=128, causal).  The central
     difference of L is the check the "Zero-th Order Algorithm for Softmax Attention
     Optimization" page builds on (提出的方法);
   * the bf16 tensor-core path against the fp32 CUDA-core path on the same bf16-valued inputs,
@@ -38,12 +40,17 @@ def _loss(cuda_lib, w, t, WQ, WK, WV):
     return float(m.loss.item())
 
 
-def test_directional_derivative_full_size_fp32(cuda_lib):
+@pytest.mark.parametrize("name", [
+    "b2_h32_n8192_d128_bf16_causal",
+    pytest.param("b1_h8_n32768_d128_bf16_causal_bounded", marks=pytest.mark.slow),
+    pytest.param("b1_h8_n131072_d128_bf16_causal_base5e5", marks=pytest.mark.slow),
+])
+def test_directional_derivative_full_size_fp32(cuda_lib, name):
     """Target E = O(W) + 0.05 noise keeps the loss small enough that its fp32 value resolves
     the change along P; P mixes the gradient direction with a random one (so the check covers
     more than the gradient's own direction); two step sizes cancel the eps^2 term of the
     central difference (Richardson)."""
-    w = W_FULL.with_sizes(dtype="f32")
+    w = WORKLOADS[name].with_sizes(dtype="f32")
     inp = make_inputs(w)
     t = to_device(inp, "f32")
     m0 = _model(cuda_lib, w, t)
@@ -73,6 +80,8 @@ def test_directional_derivative_full_size_fp32(cuda_lib):
 
     d1, d2 = central(2e-3), central(1e-3)
     fd = (4 * d2 - d1) / 3
+    print(f"\n{name}: central difference {fd:.9e}, <grad, P> {an:.9e}, "
+          f"rel {abs(fd - an) / abs(an):.3e}", flush=True)
     assert abs(fd - an) <= 1e-3 * abs(an), (fd, an, d1, d2)
 
 

@@ -5,8 +5,12 @@ synchronisation an allocation can cause, or that runs inside a component whose d
 belongs to someone else).  The library gives them one entry point that runs the whole step on
 a static scratch array inside the library instead of a caller-owned workspace.  These tests
 call it through the C ABI and check its outputs against the workspace-based entry points
-(rope_attn_fwd + rope_attn_loss_bwd), within the parity tolerances, on two calls in a row (the
-second call runs on scratch the first one left behind).
+(rope_attn_fwd + rope_attn_loss_bwd) on two calls in a row.  Before the first checked call the
+scratch is left dirty by a step on another problem (other inputs, other length, the other
+causal flag), so state that leaked from one call into the next would show.  The forward runs
+the same kernels on the same inputs, so O, lse and the loss must agree bit for bit; the weight
+gradients may differ only by the free order of the backward's fp32 reductions (and the bf16
+rounding that follows), far below the parity bars.
 
 This file is named so that pytest collects it last.
 """
@@ -18,7 +22,8 @@ from workloads import WORKLOADS, make_inputs
 
 pytestmark = pytest.mark.gpu
 
-TOL = {"f32": 1e-4, "bf16": 2e-2}
+# weight gradients: reduction order only (the parity bars are 1e-4 and 2e-2)
+DW_TOL = {"f32": 1e-5, "bf16": 2e-3}
 
 
 def _rel(a, b):
@@ -48,7 +53,17 @@ def test_noalloc_step_matches_workspace_entry_points(cuda_lib, w):
     ref.step()
     torch.cuda.synchronize()
     assert ra.last_error() == ra.RA_OK
-    tol = TOL[w.dtype]
+    # leave the scratch dirty: a step on other inputs, another length, the other causal flag
+    wd = w.with_sizes(n=w.n // 2 + 37, causal=not w.causal)
+    inpd = make_inputs(wd, seed=11)
+    td = {k: torch.from_numpy(inpd[k]).to("cuda", dt) for k in t}
+    dirty = ra.RopeAttention(td["A1"], td["A2"], td["A3"], td["WQ"], td["WK"], td["WV"],
+                             td["E"], torch.from_numpy(inpd["pos"]).cuda(), wd.causal,
+                             wd.rope_base)
+    ra.step_noalloc(dirty.prob, dirty.O, dirty.lse, dirty.loss, dirty.dWQ, dirty.dWK, dirty.dWV)
+    torch.cuda.synchronize()
+    assert ra.last_error() == ra.RA_OK
+    tol = DW_TOL[w.dtype]
     for call in range(2):
         O = torch.full_like(ref.O, float("nan"))
         lse = torch.full_like(ref.lse, float("nan"))
@@ -57,8 +72,10 @@ def test_noalloc_step_matches_workspace_entry_points(cuda_lib, w):
         ra.step_noalloc(ref.prob, O, lse, loss, *dW)
         torch.cuda.synchronize()
         assert ra.last_error() == ra.RA_OK
-        errs = {"O": _rel(O, ref.O), "lse": _rel(lse, ref.lse), "loss": _rel(loss, ref.loss),
-                "dWQ": _rel(dW[0], ref.dWQ), "dWK": _rel(dW[1], ref.dWK),
+        assert torch.equal(O, ref.O), f"call {call}: O differs"
+        assert torch.equal(lse, ref.lse), f"call {call}: lse differs"
+        assert torch.equal(loss, ref.loss), f"call {call}: loss differs"
+        errs = {"dWQ": _rel(dW[0], ref.dWQ), "dWK": _rel(dW[1], ref.dWK),
                 "dWV": _rel(dW[2], ref.dWV)}
         bad = {k: v for k, v in errs.items() if not v <= tol}
         assert not bad, f"call {call}: {errs}"
