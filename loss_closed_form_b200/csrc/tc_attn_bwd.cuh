@@ -7,8 +7,9 @@
 //   P^T    = exp(S^T / sqrt(d) - lse_i)  recomputed softmax s(x) from the stored log-sum-exp
 //   gamma^T = P^T o (beta^T - delta_i)   gamma = diag(s) beta - s s^T beta, with the row sums
 //                                        s_i^T beta_i = <l_i, O_i> = delta_i
-//   (P^T and gamma^T are written to TMEM, where they are the A operands of the next two
-//    products; gamma^T also goes to shared memory as the B operand of dQ~^T)
+//   (P^T and gamma^T are written to TMEM over the columns S^T occupied, where they are the A
+//    operands of the next two products; gamma^T also goes to shared memory as the B operand
+//    of dQ~^T, which is accumulated over the columns beta^T occupied)
 //   dV    += P^T l_i                   (accumulated in TMEM over all query tiles)
 //   dK~   += gamma^T Q~_i              (scaled by 1/sqrt(d) and un-rotated at the end)
 //   dQ~_i^T = K~^T gamma^T             (d on TMEM lanes; staged in shared memory and added to
@@ -20,6 +21,12 @@
 //
 // Definitions: "RoPE Attention kan bijna lineair worden getraind", Methodologie 1 (s, l,
 // beta, gamma) and 2 (gamma_1 = diag(s) beta, gamma_2 = s s^T beta).
+//
+// TMEM holds two step buffers of 128 columns, [S^T | beta^T] for query tiles i and i + 1
+// (i even in buffer 0), then dK~ and dV: while the softmax warps turn one buffer into P^T and
+// gamma^T, the tensor cores run the other buffer's products, and the next-but-one step's S^T
+// and beta^T are issued as soon as a buffer's products have completed and its dQ~^T has been
+// read out.
 //
 // Warp roles (448 threads): warps 0-7 softmax / gamma (two warpgroups over the same 128 key
 // rows, each taking half of the 64 query columns) and the epilogue (warps 0-3 dK, 4-7 dV),
@@ -47,15 +54,15 @@ struct BwdCfg {
   static constexpr int V_OFF = K_OFF + KTILE;
   static constexpr int Q_OFF = V_OFF + KTILE;            // NSQ stages
   static constexpr int L_OFF = Q_OFF + NSQ * QTILE;      // NSQ stages
-  static constexpr int G_OFF = L_OFF + NSQ * QTILE;      // gamma^T, B operand of dQ~^T
-  static constexpr int DQS_OFF = G_OFF + PG;              // fp32 [BQ][D] dQ~ staging tile
+  static constexpr int G_OFF = L_OFF + NSQ * QTILE;      // gamma^T [2], B operand of dQ~^T
+  static constexpr int DQS_OFF = G_OFF + 2 * PG;          // fp32 [BQ][D] dQ~ staging tile
   static constexpr int DQS = BQ * D * 4;
   // float [NSQ][BQ / 2][4]: (-lse * log2(e) of rows 2i, 2i + 1, delta of rows 2i, 2i + 1)
   static constexpr int LD_OFF = DQS_OFF + DQS;
   static constexpr int BAR_OFF = LD_OFF + NSQ * BQ * 8;
-  // kv_full, q_full[NSQ], q_empty[NSQ], s_full, s_free, pg_full, pg_free, dq_full, dq_free,
-  // acc_done, drain, dqs_full, dqs_free
-  static constexpr int NBAR = 1 + 2 * NSQ + 12;   // ... + tab_full, ep_full
+  // kv_full, q_full[NSQ], q_empty[NSQ], s_full[2], pg_full[2], pg_done[2], dq_full[2],
+  // dq_free[2], acc_done, drain, dqs_full, dqs_free, tab_full, ep_full
+  static constexpr int NBAR = 1 + 2 * NSQ + 10 + 6;
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
   static constexpr int SMEM_USED = MISC_OFF + 64;
   static constexpr int SMEM_ALLOC =
@@ -67,8 +74,10 @@ struct BwdCfg {
   static_assert(TABT <= 2 * KTILE && 2 * KTILE <= 2 * NSQ * QTILE, "epilogue staging");
   static constexpr int THREADS = 448;
   static constexpr int W_DRAIN = 8, W_PROD = 12, W_MMA = 13;
-  // TMEM columns
-  static constexpr uint32_t T_S = 0, T_B = 64, T_DQ = 128, T_PT = 192, T_GT = 224, T_DK = 256,
+  // TMEM columns: step buffer b at 128 b holds S^T (columns 0-63) and beta^T (64-127); the
+  // softmax warpgroup h then writes P^T at 32 h and gamma^T at 32 h + 16 (16 columns each, two
+  // bf16 per column) and dQ~^T is accumulated at 64
+  static constexpr uint32_t T_BUF = 128, T_B = 64, T_DQ = 64, T_GT = 16, T_DK = 256,
                             T_DV = 256 + D;
   static constexpr uint32_t T_COLS = 512;
   static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
@@ -103,18 +112,17 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
   const uint32_t b_kv = smem_u32(&bars[0]);
   auto b_qfull = [&](int s) { return smem_u32(&bars[1 + s]); };
   auto b_qempty = [&](int s) { return smem_u32(&bars[1 + C::NSQ + s]); };
-  const uint32_t b_sfull = smem_u32(&bars[1 + 2 * C::NSQ]);
-  const uint32_t b_sfree = smem_u32(&bars[2 + 2 * C::NSQ]);
-  const uint32_t b_pgfull = smem_u32(&bars[3 + 2 * C::NSQ]);
-  const uint32_t b_pgfree = smem_u32(&bars[4 + 2 * C::NSQ]);
-  const uint32_t b_dqfull = smem_u32(&bars[5 + 2 * C::NSQ]);
-  const uint32_t b_dqfree = smem_u32(&bars[6 + 2 * C::NSQ]);
-  const uint32_t b_acc = smem_u32(&bars[7 + 2 * C::NSQ]);
-  const uint32_t b_drain = smem_u32(&bars[8 + 2 * C::NSQ]);
-  const uint32_t b_dqsfull = smem_u32(&bars[9 + 2 * C::NSQ]);
-  const uint32_t b_dqsfree = smem_u32(&bars[10 + 2 * C::NSQ]);
-  const uint32_t b_tab = smem_u32(&bars[11 + 2 * C::NSQ]);  // RoPE rows of the key tile landed
-  const uint32_t b_ep = smem_u32(&bars[12 + 2 * C::NSQ]);   // dK / dV staging written
+  auto b_sfull = [&](int b) { return smem_u32(&bars[1 + 2 * C::NSQ + b]); };   // S, beta in
+  auto b_pgfull = [&](int b) { return smem_u32(&bars[3 + 2 * C::NSQ + b]); };  // P, gamma out
+  auto b_pgdone = [&](int b) { return smem_u32(&bars[5 + 2 * C::NSQ + b]); };  // products done
+  auto b_dqfull = [&](int b) { return smem_u32(&bars[7 + 2 * C::NSQ + b]); };  // dQ~^T in
+  auto b_dqfree = [&](int b) { return smem_u32(&bars[9 + 2 * C::NSQ + b]); };  // dQ~^T read
+  const uint32_t b_acc = smem_u32(&bars[11 + 2 * C::NSQ]);
+  const uint32_t b_drain = smem_u32(&bars[12 + 2 * C::NSQ]);
+  const uint32_t b_dqsfull = smem_u32(&bars[13 + 2 * C::NSQ]);
+  const uint32_t b_dqsfree = smem_u32(&bars[14 + 2 * C::NSQ]);
+  const uint32_t b_tab = smem_u32(&bars[15 + 2 * C::NSQ]);  // RoPE rows of the key tile landed
+  const uint32_t b_ep = smem_u32(&bars[16 + 2 * C::NSQ]);   // dK / dV staging written
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   // grid (heads of a group, key tile, group): the CTAs are dispatched x fastest, so each
@@ -136,12 +144,13 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       mbar_init(b_qfull(s), 2);  // TMA bytes + the staged lse / delta
       mbar_init(b_qempty(s), 1);
     }
-    mbar_init(b_sfull, 1);
-    mbar_init(b_sfree, 256);
-    mbar_init(b_pgfull, 256);
-    mbar_init(b_pgfree, 1);
-    mbar_init(b_dqfull, 1);
-    mbar_init(b_dqfree, 128);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(b_sfull(b), 1);
+      mbar_init(b_pgfull(b), 256);
+      mbar_init(b_pgdone(b), 1);
+      mbar_init(b_dqfull(b), 1);
+      mbar_init(b_dqfree(b), 128);
+    }
     mbar_init(b_acc, 1);
     mbar_init(b_drain, 1);
     mbar_init(b_dqsfull, 128);
@@ -210,6 +219,10 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     }
   } else if (warp == C::W_MMA) {
     // ------------------------------------------------------------------ MMA issuer
+    // per step i in buffer b = i % 2: dV and dK (they read P^T, gamma^T over the S^T columns),
+    // then dQ~^T_i (over the beta^T columns).  S^T of step i + 2 follows as soon as dV and dK
+    // have completed, while dQ~^T_i still runs; beta^T of step i + 2 once the drain has read
+    // dQ~^T_i, while S^T runs: the tensor pipe always has a product queued behind the wait.
     if (lane == 0) {
       constexpr uint32_t idesc_sb = idesc_bf16_f32(128, C::BQ, false, false);
       constexpr uint32_t idesc_kv = idesc_bf16_f32(128, D, false, true);
@@ -217,58 +230,73 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       // descriptor low words per buffer (sw128_lo), offsets added per K step (sw128_at)
       const uint32_t ka_k = sw128_lo(sbase + C::K_OFF, 16), va_k = sw128_lo(sbase + C::V_OFF, 16);
       const uint32_t ka_mn = sw128_lo(sbase + C::K_OFF, C::KBLK);
-      const uint32_t gt_mn = sw128_lo(sbase + C::G_OFF, C::KBLK);
       bool ok = mbar_wait(b_kv, 0, abort_flag, lim);
-      auto issue_sb = [&](int ii) -> bool {
+      // S^T (z = 0) or beta^T (z = 1) of step ii into its buffer
+      auto issue_sb = [&](int ii, int z) {
         const int s = ii % C::NSQ;
-        if (!mbar_wait(b_qfull(s), (ii / C::NSQ) & 1, abort_flag, lim)) return false;
-        tc_fence_after();
-        const uint32_t qb_k = sw128_lo(sbase + C::Q_OFF + s * C::QTILE, 16);
-        const uint32_t lb_k = sw128_lo(sbase + C::L_OFF + s * C::QTILE, 16);
+        const uint32_t ab = z ? va_k : ka_k;
+        const uint32_t bb = sw128_lo(sbase + (z ? C::L_OFF : C::Q_OFF) + s * C::QTILE, 16);
+        const uint32_t d_acc = tmem + (ii & 1) * C::T_BUF + (z ? C::T_B : 0);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t ko = (kk >> 2) * C::KBLK + (kk & 3) * 32;
           const uint32_t qo = (kk >> 2) * C::QBLK + (kk & 3) * 32;
-          mma_ss(tmem + C::T_S, sw128_at(ka_k, ko), sw128_at(qb_k, qo), idesc_sb, kk > 0);
-          mma_ss(tmem + C::T_B, sw128_at(va_k, ko), sw128_at(lb_k, qo), idesc_sb, kk > 0);
+          mma_ss(d_acc, sw128_at(ab, ko), sw128_at(bb, qo), idesc_sb, kk > 0);
         }
-        mma_commit(b_sfull);
+      };
+      auto wait_q = [&](int ii) -> bool {
+        if (!mbar_wait(b_qfull(ii % C::NSQ), (ii / C::NSQ) & 1, abort_flag, lim)) return false;
+        tc_fence_after();
         return true;
       };
       tc_fence_after();
-      if (ok) ok = issue_sb(0);
+      for (int ii = 0; ok && ii < 2 && ii < NI; ++ii) {
+        if (!(ok = wait_q(ii))) break;
+        issue_sb(ii, 0);
+        issue_sb(ii, 1);
+        mma_commit(b_sfull(ii));
+      }
       for (int ii = 0; ok && ii < NI; ++ii) {
-        if (ii + 1 < NI) {
-          if (!(ok = mbar_wait(b_sfree, ii & 1, abort_flag, lim))) break;
-          if (!(ok = issue_sb(ii + 1))) break;
-        }
-        const int s = ii % C::NSQ;
-        if (!(ok = mbar_wait(b_pgfull, ii & 1, abort_flag, lim))) break;
+        const int s = ii % C::NSQ, b = ii & 1;
+        const uint32_t ph = (ii >> 1) & 1;
+        if (!(ok = mbar_wait(b_pgfull(b), ph, abort_flag, lim))) break;
         tc_fence_after();
+        const uint32_t buf = tmem + b * C::T_BUF;
+        // dV += P^T l_i, dK += gamma^T Q~_i: M = 128 keys, N = D, K = 64 queries, with P^T and
+        // gamma^T read from TMEM (two bf16 per column, 8 columns per K step of 16 queries:
+        // queries 16 kk .. of warpgroup kk / 2 at 32 (kk / 2) + 8 (kk % 2))
         const uint32_t qb_mn = sw128_lo(sbase + C::Q_OFF + s * C::QTILE, C::QBLK);
         const uint32_t lb_mn = sw128_lo(sbase + C::L_OFF + s * C::QTILE, C::QBLK);
-        // dV += P^T l_i, dK += gamma^T Q~_i: M = 128 keys, N = D, K = 64 queries, with
-        // P^T and gamma^T read from TMEM (two bf16 per column, 8 columns per K step)
 #pragma unroll
         for (int kk = 0; kk < C::BQ / 16; ++kk) {
-          mma_ts(tmem + C::T_DV, tmem + C::T_PT + kk * 8, sw128_at(lb_mn, kk * 2048), idesc_kv,
-                 (ii > 0 || kk > 0));
-          mma_ts(tmem + C::T_DK, tmem + C::T_GT + kk * 8, sw128_at(qb_mn, kk * 2048), idesc_kv,
+          const uint32_t pa = buf + 32 * (kk >> 1) + 8 * (kk & 1);
+          mma_ts(tmem + C::T_DV, pa, sw128_at(lb_mn, kk * 2048), idesc_kv, (ii > 0 || kk > 0));
+          mma_ts(tmem + C::T_DK, pa + C::T_GT, sw128_at(qb_mn, kk * 2048), idesc_kv,
                  (ii > 0 || kk > 0));
         }
-        // dQ~_i^T = K~^T gamma^T   (M = D, N = 64 queries, K = 128 keys), once the drain has
-        // read the previous tile's dQ~ out of TMEM
-        if (ii > 0) {
-          if (!(ok = mbar_wait(b_dqfree, (ii - 1) & 1, abort_flag, lim))) break;
-          tc_fence_after();
-        }
+        mma_commit(b_pgdone(b));
+        mma_commit(b_qempty(s));
+        // dQ~_i^T = K~^T gamma^T (M = D, N = 64 queries, K = 128 keys) over the columns beta^T
+        // held (the softmax warps have read them)
+        const uint32_t gt_mn = sw128_lo(sbase + C::G_OFF + b * C::PG, C::KBLK);
 #pragma unroll
         for (int kk = 0; kk < C::BK / 16; ++kk)
-          mma_ss(tmem + C::T_DQ, sw128_at(ka_mn, kk * 2048), sw128_at(gt_mn, kk * 2048),
-                 idesc_dq, kk > 0);
-        mma_commit(b_dqfull);
-        mma_commit(b_pgfree);
-        mma_commit(b_qempty(s));
+          mma_ss(buf + C::T_DQ, sw128_at(ka_mn, kk * 2048), sw128_at(gt_mn, kk * 2048), idesc_dq,
+                 kk > 0);
+        mma_commit(b_dqfull(b));
+        if (ii + 2 < NI) {
+          // S^T_i+2 over P^T, gamma^T once dV and dK have read them; beta^T_i+2 over dQ~^T_i
+          // once the drain has read it (gamma^T slot b, read by dQ~^T_i, is rewritten only
+          // after sfull, which follows beta^T)
+          if (!(ok = wait_q(ii + 2))) break;
+          if (!(ok = mbar_wait(b_pgdone(b), ph, abort_flag, lim))) break;
+          tc_fence_after();
+          issue_sb(ii + 2, 0);
+          if (!(ok = mbar_wait(b_dqfree(b), ph, abort_flag, lim))) break;
+          tc_fence_after();
+          issue_sb(ii + 2, 1);
+          mma_commit(b_sfull(b));
+        }
       }
       if (ok) {
         mma_commit(b_acc);
@@ -287,17 +315,17 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     bool ok = true;
     for (int ii = 0; ii < NI; ++ii) {
       const int q0 = (i_start + ii) * C::BQ;
-      const int stg = ii % C::NSQ;
+      const int stg = ii % C::NSQ, b = ii & 1;
       // the stage's lse / delta (and S^T, beta^T below) for this query tile
       if (!(ok = mbar_wait_warp(b_qfull(stg), (ii / C::NSQ) & 1, abort_flag, lim))) break;
-      if (!(ok = mbar_wait_warp(b_sfull, ii & 1, abort_flag, lim))) break;
+      if (!(ok = mbar_wait_warp(b_sfull(b), (ii >> 1) & 1, abort_flag, lim))) break;
       tc_fence_after();
+      // this warpgroup's 32 query columns of S^T and beta^T in step buffer b
+      const uint32_t buf = tmem + lane_base + b * C::T_BUF + 32 * half;
       uint32_t sr[32], br[32];
-      tmem_ld32(tmem + lane_base + C::T_S + 32 * half, sr);
-      tmem_ld32(tmem + lane_base + C::T_B + 32 * half, br);
+      tmem_ld32(buf, sr);
+      tmem_ld32(buf + C::T_B, br);
       tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive(b_sfree);
       const uint32_t ld_row = sbase + C::LD_OFF + (stg * C::BQ + 32 * half) * 8;
       const int qh = q0 + 32 * half;
       const bool full = key < n && qh + 32 <= n && (!p.causal || key <= qh);
@@ -331,14 +359,12 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
           gw[h] &= keep;
         }
       }
-      // the previous tile's products have read P^T, gamma^T (TMEM) and gamma^T (smem)
-      if (ii > 0) {
-        if (!(ok = mbar_wait_warp(b_pgfree, (ii - 1) & 1, abort_flag, lim))) break;
-        tc_fence_after();
-      }
-      tmem_st16(tmem + lane_base + C::T_PT + 16 * half, pw);
-      tmem_st16(tmem + lane_base + C::T_GT + 16 * half, gw);
-      const uint32_t gsm = sbase + C::G_OFF;
+      // P^T and gamma^T over the S^T columns this warpgroup has just read (the products of
+      // step i - 2, which read this buffer and gamma^T slot b, completed before S^T of step i
+      // was issued)
+      tmem_st16(buf, pw);
+      tmem_st16(buf + C::T_GT, gw);
+      const uint32_t gsm = sbase + C::G_OFF + b * C::PG;
 #pragma unroll
       for (int c8 = 0; c8 < 4; ++c8)
         st_shared_v4(gsm + sw128_offset(row, 4 * half + c8), gw[4 * c8], gw[4 * c8 + 1],
@@ -346,7 +372,7 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       tmem_wait_st();
       fence_proxy_async_smem();
       tc_fence_before();
-      mbar_arrive(b_pgfull);
+      mbar_arrive(b_pgfull(b));
     }
     // ---- dK = rot^-1(scale * sum gamma^T Q~) (warps 0-3), dV = sum P^T l (warps 4-7):
     //      one key row per thread.  Once every product has completed, K~, V and the query
@@ -417,15 +443,16 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     const uint32_t stage = sbase + C::DQS_OFF;
     const bool issuer = tid == 32 * C::W_DRAIN;
     for (int ii = 0; ii < NI; ++ii) {
-      if (!mbar_wait_warp(b_dqfull, ii & 1, abort_flag, lim)) break;
+      const int b = ii & 1;
+      if (!mbar_wait_warp(b_dqfull(b), (ii >> 1) & 1, abort_flag, lim)) break;
       tc_fence_after();
       uint32_t r0[32], r1[32];
-      const uint32_t dq = tmem + lane_base + C::T_DQ;
+      const uint32_t dq = tmem + lane_base + b * C::T_BUF + C::T_DQ;
       tmem_ld32(dq, r0);
       tmem_ld32(dq + 32, r1);
       tmem_wait_ld();
       tc_fence_before();
-      mbar_arrive(b_dqfree);
+      mbar_arrive(b_dqfree(b));
       // the staging tile is free once the previous bulk reduction has read it
       if (!mbar_wait_warp(b_dqsfree, (ii & 1) ^ 1, abort_flag, lim)) break;
       if (has_row) {
