@@ -45,8 +45,8 @@ struct FwdCfg {
   static constexpr int V_OFF = K_OFF + NS * TILE;
   static constexpr int BAR_OFF = V_OFF + NS * TILE;
   // barriers: q_full, k_full[NS], k_empty[NS], v_full[NS], v_empty[NS], s_full[2],
-  //           p_full[2], pv_done[2], drain, e_full[2]
-  static constexpr int NBAR = 1 + 4 * NS + 6 + 1 + 2;
+  //           p_full[2], pv_done[2], drain, e_full[2], s_free[2]
+  static constexpr int NBAR = 1 + 4 * NS + 6 + 1 + 2 + 2;
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;  // tmem slot, abort flag
   static constexpr int SMEM_USED = MISC_OFF + 16;
   // at least half of the SM's shared memory: one CTA per SM, so the 512-column TMEM
@@ -58,8 +58,14 @@ struct FwdCfg {
   // exceed the 384 x 168 the CTA is launched with
   static constexpr int REG_SOFTMAX = 216, REG_OTHER = 64;
   static_assert(256 * REG_SOFTMAX + 128 * REG_OTHER <= 384 * 168, "register hand-over");
-  // TMEM columns: S_t at 128 t (P_t over its first 64 columns), O_t at 256 + 128 t
-  static constexpr uint32_t T_S0 = 0, T_O0 = 256, T_COLS = 512;
+  // TMEM columns: S_t at 128 t, O_t at 256 + O_STRIDE t.  With D = 128 the four take all 512
+  // columns and P_t is written over the first 64 columns of S_t; with D = 64 each O_t takes 64
+  // columns and P_t gets its own 64 at 384 + 64 t (SEP_P), so S_t,j+1 need not wait for the
+  // product that reads P_t,j
+  static constexpr bool SEP_P = D == 64;
+  static constexpr uint32_t O_STRIDE = SEP_P ? D : 128;
+  static constexpr uint32_t T_S0 = 0, T_O0 = 256, T_P0 = 384, T_COLS = 512;
+  static_assert(!SEP_P || T_O0 + 2 * O_STRIDE <= T_P0, "TMEM plan");
   // loss partial sums written per query tile (one per softmax warp)
   static constexpr int LOSS_PARTS = 4;
 };
@@ -105,6 +111,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
   auto b_pvdone = [&](int t) { return smem_u32(&bars[5 + 4 * C::NS + t]); };
   const uint32_t b_drain = smem_u32(&bars[7 + 4 * C::NS]);
   auto b_efull = [&](int t) { return smem_u32(&bars[8 + 4 * C::NS + t]); };  // E tile landed
+  auto b_sfree = [&](int t) { return smem_u32(&bars[10 + 4 * C::NS + t]); };  // S_t read (SEP_P)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   // grid (heads of a group, pair rank, group): the CTAs are dispatched x fastest, so each
@@ -133,6 +140,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
       mbar_init(b_sfull(t), 1);
       mbar_init(b_pfull(t), 4);  // one arrival per softmax warp
       mbar_init(b_pvdone(t), 1);
+      mbar_init(b_sfree(t), 4);  // one arrival per softmax warp
     }
     mbar_init(b_drain, 1);
     mbar_init(b_efull(0), 1);
@@ -209,12 +217,12 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
         mma_commit(b_sfull(t));
       };
       auto issue_pv = [&](int t, int j) {
-        const uint32_t pa = tmem + C::T_S0 + 128 * t;
+        const uint32_t pa = tmem + (C::SEP_P ? C::T_P0 + 64 * t : C::T_S0 + 128 * t);
         const uint32_t vb = sw128_lo(sbase + C::V_OFF + (j % C::NS) * C::TILE, C::BLK);
 #pragma unroll
         for (int kk = 0; kk < C::BN / 16; ++kk)
-          mma_ts(tmem + C::T_O0 + 128 * t, pa + kk * 8, sw128_at(vb, kk * 2048), idesc_pv,
-                 (j > 0 || kk > 0));
+          mma_ts(tmem + C::T_O0 + C::O_STRIDE * t, pa + kk * 8, sw128_at(vb, kk * 2048),
+                 idesc_pv, (j > 0 || kk > 0));
         mma_commit(b_pvdone(t));
       };
       bool ok = mbar_wait(b_q, 0, abort_flag, lim);
@@ -225,34 +233,63 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
         issue_s(1, 0);
         mma_commit(b_kempty(0));
       }
-      for (int j = 0; ok && j < T1; ++j) {
-        const int s = j % C::NS;
-        const bool next0 = j + 1 < T0, next1 = j + 1 < T1;
-        if (!(ok = mbar_wait(b_vfull(s), (j / C::NS) & 1, abort_flag, lim))) break;
-        if (j < T0) {
-          if (!(ok = mbar_wait(b_pfull(0), j & 1, abort_flag, lim))) break;
-          tc_fence_after();
-          issue_pv(0, j);
+      if constexpr (C::SEP_P) {
+        // per key tile j: S_t,j+1 as soon as softmax t has read S_t,j, then P_t,j V_j once
+        // softmax t has written P_t,j (its own columns: no wait on the previous product)
+        for (int j = 0; ok && j < T1; ++j) {
+          if (j + 1 < T1) {
+            const int s1 = (j + 1) % C::NS;
+            if (!(ok = mbar_wait(b_kfull(s1), ((j + 1) / C::NS) & 1, abort_flag, lim))) break;
+            for (int t = 0; ok && t < 2; ++t) {
+              if (j + 1 >= (t ? T1 : T0)) continue;
+              if (!(ok = mbar_wait(b_sfree(t), j & 1, abort_flag, lim))) break;
+              tc_fence_after();
+              issue_s(t, j + 1);
+            }
+            if (!ok) break;
+            mma_commit(b_kempty(s1));
+          }
+          const int s = j % C::NS;
+          if (!(ok = mbar_wait(b_vfull(s), (j / C::NS) & 1, abort_flag, lim))) break;
+          for (int t = 0; ok && t < 2; ++t) {
+            if (j >= (t ? T1 : T0)) continue;
+            if (!(ok = mbar_wait(b_pfull(t), j & 1, abort_flag, lim))) break;
+            tc_fence_after();
+            issue_pv(t, j);
+          }
+          if (!ok) break;
+          mma_commit(b_vempty(s));
         }
-        if (next1) {
-          const int s1 = (j + 1) % C::NS;
-          if (!(ok = mbar_wait(b_kfull(s1), ((j + 1) / C::NS) & 1, abort_flag, lim))) break;
-        }
-        if (next0) {
-          // S_0,j+1 overwrites P_0,j: wait until the product reading it has completed
-          if (!(ok = mbar_wait(b_pvdone(0), j & 1, abort_flag, lim))) break;
+      } else {
+        for (int j = 0; ok && j < T1; ++j) {
+          const int s = j % C::NS;
+          const bool next0 = j + 1 < T0, next1 = j + 1 < T1;
+          if (!(ok = mbar_wait(b_vfull(s), (j / C::NS) & 1, abort_flag, lim))) break;
+          if (j < T0) {
+            if (!(ok = mbar_wait(b_pfull(0), j & 1, abort_flag, lim))) break;
+            tc_fence_after();
+            issue_pv(0, j);
+          }
+          if (next1) {
+            const int s1 = (j + 1) % C::NS;
+            if (!(ok = mbar_wait(b_kfull(s1), ((j + 1) / C::NS) & 1, abort_flag, lim))) break;
+          }
+          if (next0) {
+            // S_0,j+1 overwrites P_0,j: wait until the product reading it has completed
+            if (!(ok = mbar_wait(b_pvdone(0), j & 1, abort_flag, lim))) break;
+            tc_fence_after();
+            issue_s(0, j + 1);
+          }
+          if (!(ok = mbar_wait(b_pfull(1), j & 1, abort_flag, lim))) break;
           tc_fence_after();
-          issue_s(0, j + 1);
-        }
-        if (!(ok = mbar_wait(b_pfull(1), j & 1, abort_flag, lim))) break;
-        tc_fence_after();
-        issue_pv(1, j);
-        mma_commit(b_vempty(s));
-        if (next1) {
-          if (!(ok = mbar_wait(b_pvdone(1), j & 1, abort_flag, lim))) break;
-          tc_fence_after();
-          issue_s(1, j + 1);
-          mma_commit(b_kempty((j + 1) % C::NS));
+          issue_pv(1, j);
+          mma_commit(b_vempty(s));
+          if (next1) {
+            if (!(ok = mbar_wait(b_pvdone(1), j & 1, abort_flag, lim))) break;
+            tc_fence_after();
+            issue_s(1, j + 1);
+            mma_commit(b_kempty((j + 1) % C::NS));
+          }
         }
       }
       if (!ok) {
@@ -271,7 +308,9 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
     const int Tt = t ? T1 : T0;
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t s_col = tmem + lane_base + C::T_S0 + 128 * t;
-    const uint32_t o_col = tmem + lane_base + C::T_O0 + 128 * t;
+    const uint32_t o_col = tmem + lane_base + C::T_O0 + C::O_STRIDE * t;
+    // P_t: over the first 64 columns of S_t, or its own columns (SEP_P)
+    const uint32_t p_col = C::SEP_P ? tmem + lane_base + C::T_P0 + 64 * t : s_col;
     float m = -INFINITY, l = 0.f;
     bool ok = true;
     for (int j = 0; j < Tt; ++j) {
@@ -288,6 +327,11 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
         reg_fence32(xr[c]);
 #pragma unroll
         for (int i = 0; i < 32; ++i) x[32 * c + i] = __uint_as_float(xr[c][i]);
+      }
+      if constexpr (C::SEP_P) {
+        // S_t is in registers: the MMA warp may compute S_t,j+1 into its columns now
+        tc_fence_before();
+        mbar_arrive_warp(b_sfree(t));
       }
       const int key0 = j * C::BN;
       if (key0 + C::BN > n || (p.causal && j == qt)) {
@@ -309,13 +353,22 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
 #pragma unroll
       for (int k = 0; k < 4; ++k) mt[k] = fmaxf(mt[k], x[124 + k]);
       const float mnew = fmaxf(m, fmax3f(mt[0], mt[1], fmaxf(mt[2], mt[3])) * p.scale_log2);
+      if constexpr (C::SEP_P) {
+        // the product P_t,j-1 V_j-1 has completed before P_t,j is written over P_t,j-1 and O_t
+        // may be rescaled (S_t,j no longer implies it)
+        if (j > 0) {
+          if (!(ok = mbar_wait_warp(b_pvdone(t), (j - 1) & 1, abort_flag, lim))) break;
+          tc_fence_after();
+        }
+      }
       if (j == 0) {
         m = mnew;
       } else {
         const bool need = mnew > m + 8.f;
         if (__any_sync(0xffffffffu, need)) {
-          // S_t,j was issued after the product of tile j - 1 completed, and its commit
-          // covers that product: O_t is final for tiles < j and can be rescaled in place
+          // O_t is final for tiles < j (D = 128: S_t,j was issued after the product of tile
+          // j - 1 completed and its commit covers that product; SEP_P: waited for above) and
+          // can be rescaled in place
           const float alpha = need ? ex2(m - mnew) : 1.f;
           if (need) {
             l *= alpha;
@@ -344,7 +397,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
           ps1 += p1;
           pk[i] = pack_bf16x2(p0, p1);
         }
-        tmem_st16(s_col + 16 * c, pk);
+        tmem_st16(p_col + 16 * c, pk);
       }
       l += ps0 + ps1;
       tmem_wait_st();
