@@ -51,6 +51,8 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-input-grads", action="store_true")
+    ap.add_argument("--approx", action="store_true",
+                    help="also time the near-linear approximate method (rope_attn_approx_step)")
     return ap.parse_args()
 
 
@@ -306,6 +308,39 @@ def run_ours(args, rank, world, local_rank):
                 ms_ig, n_ig = prof_ig[kname]
                 input_grads = {"kernel": kname, "avg_launch_ms": round(ms_ig / max(1, n_ig), 4)}
 
+    # ---- the near-linear approximate method (rope_attn_approx_step), timed on its own -----
+    approx = None
+    if args.approx:
+        prob = m.prob
+        f32 = dict(dtype=torch.float32, device=dev)
+        ao = {"O": torch.empty_like(m.O), "loss": torch.zeros((), **f32),
+              **{k: torch.empty_like(m.dWQ) for k in ("dWQ", "dWK", "dWV")}}
+        aws = torch.empty(ra.approx_workspace_bytes(prob), dtype=torch.uint8, device=dev)
+
+        def astep():
+            ra.approx_step(prob, ao["O"], ao["loss"], ao["dWQ"], ao["dWK"], ao["dWV"], aws)
+        astep()
+        torch.cuda.synchronize(dev)
+        reps = 3
+        ra.profile_read()
+        ra.profile_enable(True)
+        e0.record(stream)
+        for _ in range(reps):
+            astep()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        prof_ap = ra.profile_read()
+        ra.profile_enable(False)
+        st = ra.last_error()
+        if st != ra.RA_OK:
+            raise RuntimeError(f"kernel status after the approximate run: {ra.status_string(st)}")
+        approx = {"ms_per_step": round(e0.elapsed_time(e1) / reps, 3),
+                  "exact_ms_per_step": round(ms_max / args.steps, 4),
+                  "workspace_bytes": int(aws.numel()), "degree": 1,
+                  "kernels": {k: round(v[0] / reps, 3) for k, v in
+                              sorted(prof_ap.items(), key=lambda kv: -kv[1][0])}}
+        del aws
+
     if rank != 0:
         return None
 
@@ -337,6 +372,8 @@ def run_ours(args, rank, world, local_rank):
         "e2e": e2e,
         "peaks_source": src,
     }
+    if approx is not None:
+        line["approx"] = approx
     if input_grads is not None:
         line["input_grads"] = dict(input_grads, **(kernel_roofline(
             w, input_grads["kernel"], input_grads["avg_launch_ms"], pk) or {}))

@@ -150,6 +150,29 @@ ra_status rope_attn_combined_grad(const float* dWK, int32_t H, int32_t d, float*
                                   void* stream);
 
 /*
+ * The near-linear approximate method of "RoPE Attention kan bijna lineair worden getraind"
+ * (Methodologie 2 "Low-Rank Benaderingsstrategie"; Resultaten, Theorem 5.7), with the degree-1
+ * polynomial method: on bounded scores exp(z) is replaced by 1 + z = U_i . F_j with the d + 1
+ * features U_i = (1, d^-1/4 q~_i), F_j = (1, d^-1/4 k~_j), so s~ = U F^T normalised per row is the
+ * low-rank U1 V1^T; gamma_1 = diag(s~) beta is contracted through row-wise Kronecker products
+ * of the factors with [l, -delta] and [v, 1], gamma_2 through the precomputed delta = <l, O>.
+ * Causal masks use exclusive prefix / suffix sums of the low-rank states over chunks of 256 rows
+ * and the pairs inside a chunk directly; work and memory are linear in n.  All arithmetic is
+ * fp32 on the CUDA cores (inputs of either dtype).  The result approximates the exact one:
+ * its accuracy depends on the bound of the scores (the method's bounded-entry regime).
+ *   O           : device [B][H][n][d], element type p->dtype (written): s~ V
+ *   loss        : device fp32 scalar 1/2 ||O - E||^2 (written; may be NULL)
+ *   dWQ/dWK/dWV : device [H][d][d] fp32 (overwritten): the approximate weight gradients
+ *   ws          : device workspace of rope_attn_approx_workspace_bytes(p) bytes (256-byte
+ *                 aligned); it grows as n (d + 1)^2 d / 64 floats for the chunk states plus
+ *                 ten [B][H][n][d] fp32 arrays
+ * p->E must not be NULL.  Validation and errors as the other entry points.
+ */
+size_t rope_attn_approx_workspace_bytes(const ra_problem* p);
+ra_status rope_attn_approx_step(const ra_problem* p, void* O, float* loss, float* dWQ, float* dWK,
+                                float* dWV, void* ws, size_t ws_bytes, void* stream);
+
+/*
  * Synchronises `stream`, then reports and clears the device-side status word of the current
  * device: RA_ERR_TIMEOUT if a kernel gave up waiting since the last call, else RA_OK
  * (RA_ERR_CUDA if the synchronisation itself failed).

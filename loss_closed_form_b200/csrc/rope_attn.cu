@@ -20,6 +20,7 @@
 #include "tc_attn_fwd.cuh"
 #include "tc_attn_bwd.cuh"
 #include "tc_proj_dw.cuh"
+#include "approx_kernels.cuh"
 
 namespace {
 
@@ -46,6 +47,11 @@ enum KernelId : int {
   K_COMB_G,
   K_PROJ_SIMT_BWD,  // launches made by a backward call (skipped on the device when the
   K_PROJ_TC_BWD,    // workspace holds this problem's intermediates)
+  K_APX_LOCAL,      // the approximate method's kernels
+  K_APX_SCAN,
+  K_APX_APPLY,
+  K_APX_INTRA,
+  K_APX_ROWS,
   K_COUNT
 };
 const char* const kKernelNames[K_COUNT] = {
@@ -53,7 +59,8 @@ const char* const kKernelNames[K_COUNT] = {
     "attn_bwd_simt", "dw_partial_simt", "dw_reduce", "loss_finalize",
     "attn_fwd_tc", "attn_bwd_tc", "proj_rope_tc", "dq_unrotate", "dw_tc",
     "input_grads_tc", "input_grads_simt", "combined_weights", "combined_grad",
-    "proj_rope_simt_bwd", "proj_rope_tc_bwd"};
+    "proj_rope_simt_bwd", "proj_rope_tc_bwd", "approx_local_sum", "approx_scan", "approx_apply",
+    "approx_intra", "approx_rows"};
 
 struct ProfRecord {
   int id;
@@ -736,6 +743,204 @@ ra_status tc_bwd(const ra_problem* p, const void* O, const float* lse, float* lo
 }
 
 // ---------------------------------------------------------------------------------------
+// The near-linear approximate method (degree-1 polynomial, low-rank states; fp32 on the CUDA
+// cores).  Workspace: RoPE table, fp32 Q~, K~, V and dQ~, dK~, dV of every instance, the loss
+// partials, the weight-gradient partials, and per-instance buffers reused instance by instance
+// (row vectors and the chunk states).
+// ---------------------------------------------------------------------------------------
+struct ApproxLayout {
+  size_t rope, qt, kt, v, dqt, dkt, dv, loss_part, dw_part;
+  size_t nd, ell, dn, delta, xq, xk, invd, sq, yv, small, big;
+  size_t total;
+  int nch, nrb, nsplit, chunk;
+};
+
+ApproxLayout make_approx_layout(const ra_problem* p) {
+  ApproxLayout L{};
+  const size_t B = p->B, H = p->H, n = p->n, d = p->d;
+  const size_t act = B * H * n * d;
+  L.nch = (int)((n + ra::approx::kChunk - 1) / ra::approx::kChunk);
+  L.nrb = (int)((n + 31) / 32);
+  const long rows = (long)B * p->n;
+  long ns = (4 * 148 + 3 * p->H - 1) / (3 * p->H);
+  ns = ns < 1 ? 1 : ns;
+  const long maxs = (rows + 63) / 64;
+  if (ns > maxs) ns = maxs;
+  L.nsplit = (int)ns;
+  L.chunk = (int)((rows + ns - 1) / ns);
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    size_t o = off;
+    off = align_up(off + bytes, kAlignWs);
+    return o;
+  };
+  L.rope = take(n * (d / 2) * sizeof(float2));
+  L.qt = take(act * 4);
+  L.kt = take(act * 4);
+  L.v = take(act * 4);
+  L.dqt = take(act * 4);
+  L.dkt = take(act * 4);
+  L.dv = take(act * 4);
+  L.loss_part = take(B * H * (size_t)L.nrb * sizeof(double));
+  L.dw_part = take(3 * H * (size_t)L.nsplit * d * d * 4);
+  L.nd = take(n * (d + 1) * 4);
+  L.ell = take(n * d * 4);
+  L.dn = take(n * 4);
+  L.delta = take(n * 4);
+  L.xq = take(n * (d + 1) * 4);
+  L.xk = take(n * (d + 1) * 4);
+  L.invd = take(n * 4);
+  L.sq = take(n * 4);
+  L.yv = take(n * (d + 1) * 4);
+  L.small = take((size_t)L.nch * (d + 1) * (d + 1) * 4);
+  L.big = take((size_t)L.nch * (d + 1) * (d + 1) * d * 4);
+  L.total = off;
+  return L;
+}
+
+template <int D, bool KRON, int W>
+void apx_state(const float* X, const float* x, const float* xs, const float* y, float* S, int n,
+               int nch, int mode, cudaStream_t st) {
+  using namespace ra::approx;
+  const float c4 = powf((float)D, -0.25f);
+  {
+    Launch l(K_APX_LOCAL, st);
+    local_sum_kernel<D, KRON, W><<<dim3(nch, 1, KRON ? D + 1 : 1), kThreads, 0, st>>>(
+        X, x, xs, y, S, n, c4);
+  }
+  const long long size = (long long)(KRON ? D + 1 : 1) * (D + 1) * W;
+  Launch l(K_APX_SCAN, st);
+  state_scan_kernel<<<(unsigned)((size + 255) / 256), 256, 0, st>>>(S, size, nch, mode);
+}
+
+template <int D, bool KRON, int W>
+void apx_apply(const float* X, const float* x, const float* ss, const float* S, float* out, int n,
+               float scale, cudaStream_t st) {
+  using namespace ra::approx;
+  constexpr int NU = D + 1;
+  const size_t smem = (size_t)(kRowBlk * (D + 1) + (KRON ? kRowBlk * (NU + 1) : 0) + NU * kEBlk) * 4;
+  auto k = apply_kernel<D, KRON, W>;
+  cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  Launch l(K_APX_APPLY, st);
+  k<<<dim3((n + kRowBlk - 1) / kRowBlk, (W + kEBlk - 1) / kEBlk), kThreads, smem, st>>>(
+      X, x, ss, S, out, n, powf((float)D, -0.25f), scale);
+}
+
+template <int D, bool FWD>
+void apx_intra(const float* Qt, const float* Kt, const float* V, const float* ell, const float* dn,
+               const float* delta, float* nd, float* dqt, float* dkt, float* dv, int n, int nch,
+               cudaStream_t st) {
+  using namespace ra::approx;
+  constexpr int NT = kChunk / kIT;
+  const size_t smem = (size_t)(4 * kIT * (D + 1) + 2 * kIT * (kIT + 1)) * 4;
+  auto k = intra_kernel<D, FWD>;
+  cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  Launch l(K_APX_INTRA, st);
+  k<<<dim3(NT * (NT + 1) / 2, nch), kThreads, smem, st>>>(Qt, Kt, V, ell, dn, delta, nd, dqt, dkt,
+                                                         dv, n, 1.0f / sqrtf((float)D));
+}
+
+template <class T, int D>
+ra_status approx_step(const ra_problem* p, void* O, float* loss, float* dWQ, float* dWK,
+                      float* dWV, void* ws, cudaStream_t st) {
+  using namespace ra::approx;
+  const ApproxLayout L = make_approx_layout(p);
+  const int n = p->n, BH = p->B * p->H;
+  const size_t nd_ = (size_t)n * D;
+  float2* tab = at<float2>(ws, L.rope);
+  {
+    const long long total = (long long)n * (D / 2);
+    const long long want = (total + 255) / 256, cap = 8LL * num_sms();
+    Launch l(K_ROPE_TABLE, st);
+    ra::simt::rope_table_kernel<<<(unsigned)(want < cap ? want : cap), 256, 0, st>>>(
+        tab, p->pos, n, D / 2, p->rope_base);
+  }
+  {
+    using namespace ra::simt;
+    size_t smem = (size_t)(kRows * (D + 4) + D * D) * sizeof(float);
+    auto k = proj_rope_kernel<T, float>;
+    cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    dim3 grid((n + kRows - 1) / kRows, BH, 3);
+    Launch l(K_PROJ_SIMT, st);
+    k<<<grid, ra::simt::kThreads, smem, st>>>(
+        (const T*)p->A1, (const T*)p->A2, (const T*)p->A3, (const T*)p->WQ, (const T*)p->WK,
+        (const T*)p->WV, tab, at<float>(ws, L.qt), at<float>(ws, L.kt), at<float>(ws, L.v), p->H,
+        n, D, ra::WsGate{nullptr, 0, 0});
+  }
+  const size_t act_bytes = (size_t)BH * nd_ * 4;
+  if (cudaMemsetAsync(at<float>(ws, L.dqt), 0, act_bytes, st) != cudaSuccess ||
+      cudaMemsetAsync(at<float>(ws, L.dkt), 0, act_bytes, st) != cudaSuccess ||
+      cudaMemsetAsync(at<float>(ws, L.dv), 0, act_bytes, st) != cudaSuccess)
+    return RA_ERR_CUDA;
+  const int mode_pre = p->causal ? 0 : 2, mode_suf = p->causal ? 1 : 2;
+  const float isd = 1.0f / sqrtf((float)D);
+  float *nd = at<float>(ws, L.nd), *ell = at<float>(ws, L.ell), *dn = at<float>(ws, L.dn),
+        *delta = at<float>(ws, L.delta), *xq = at<float>(ws, L.xq), *xk = at<float>(ws, L.xk),
+        *invd = at<float>(ws, L.invd), *sq = at<float>(ws, L.sq), *yv = at<float>(ws, L.yv),
+        *small = at<float>(ws, L.small), *big = at<float>(ws, L.big);
+  for (int bh = 0; bh < BH; ++bh) {
+    const float* Q = at<float>(ws, L.qt) + bh * nd_;
+    const float* K = at<float>(ws, L.kt) + bh * nd_;
+    const float* V = at<float>(ws, L.v) + bh * nd_;
+    float* dQ = at<float>(ws, L.dqt) + bh * nd_;
+    float* dK = at<float>(ws, L.dkt) + bh * nd_;
+    float* dV = at<float>(ws, L.dv) + bh * nd_;
+    {
+      const long long e = (long long)n * (D + 1);
+      Launch l(K_APX_ROWS, st);
+      ext_rows_kernel<<<(unsigned)((e + 255) / 256), 256, 0, st>>>(V, yv, n, D);
+    }
+    // forward: [N_i, D_i] = U_i . sum_j F_j^T [v_j, 1] (keys before the chunk) + the chunk's pairs
+    apx_state<D, false, D + 1>(K, nullptr, nullptr, yv, small, n, L.nch, mode_pre, st);
+    if (cudaMemsetAsync(nd, 0, (size_t)n * (D + 1) * 4, st) != cudaSuccess) return RA_ERR_CUDA;
+    apx_apply<D, false, D + 1>(Q, nullptr, nullptr, small, nd, n, 1.f, st);
+    if (p->causal)
+      apx_intra<D, true>(Q, K, V, nullptr, nullptr, nullptr, nd, nullptr, nullptr, nullptr, n,
+                         L.nch, st);
+    {
+      Launch l(K_APX_ROWS, st);
+      finish_fwd_kernel<T><<<L.nrb, kThreads, 0, st>>>(
+          nd, (const T*)p->E + bh * nd_, (T*)O + bh * nd_, ell, dn, delta, xq, xk, invd, sq,
+          at<double>(ws, L.loss_part) + (size_t)bh * L.nrb, n, D, isd);
+    }
+    // dQ~_i = (U_i (x) [l_i, -delta_i]) . sum_j (F_j (x) [v_j, 1])^T k~_j / (sqrt(d) D_i)
+    apx_state<D, true, D>(K, yv, nullptr, K, big, n, L.nch, mode_pre, st);
+    apx_apply<D, true, D>(Q, xq, sq, big, dQ, n, 1.f, st);
+    // dK~_j = (F_j (x) [v_j, 1]) . sum_i (U_i (x) [l_i, -delta_i] / D_i)^T q~_i / sqrt(d)
+    apx_state<D, true, D>(Q, xk, nullptr, Q, big, n, L.nch, mode_suf, st);
+    apx_apply<D, true, D>(K, yv, nullptr, big, dK, n, isd, st);
+    // dV_j = F_j . sum_i U_i^T l_i / D_i
+    apx_state<D, false, D>(Q, nullptr, invd, ell, small, n, L.nch, mode_suf, st);
+    apx_apply<D, false, D>(K, nullptr, nullptr, small, dV, n, 1.f, st);
+    if (p->causal)
+      apx_intra<D, false>(Q, K, V, ell, dn, delta, nullptr, dQ, dK, dV, n, L.nch, st);
+  }
+  {
+    using namespace ra::simt;
+    size_t smem = (size_t)2 * 16 * D * sizeof(float);
+    dim3 grid(L.nsplit, 3, p->H);
+    {
+      Launch l(K_DW_PART_SIMT, st);
+      dw_partial_kernel<T, float><<<grid, ra::simt::kThreads, smem, st>>>(
+          (const T*)p->A1, (const T*)p->A2, (const T*)p->A3, at<float>(ws, L.dqt),
+          at<float>(ws, L.dkt), at<float>(ws, L.dv), tab, at<float>(ws, L.dw_part), p->B, p->H,
+          n, D, L.chunk);
+    }
+    size_t total = (size_t)3 * p->H * D * D;
+    Launch l(K_DW_REDUCE, st);
+    dw_reduce_kernel<<<(unsigned)((total + 255) / 256), 256, 0, st>>>(
+        at<float>(ws, L.dw_part), dWQ, dWK, dWV, p->H, D, L.nsplit, nullptr, 0, 0u);
+  }
+  if (loss) {
+    Launch l(K_LOSS, st);
+    ra::simt::loss_finalize_kernel<<<1, 1024, 0, st>>>(at<double>(ws, L.loss_part), BH * L.nrb,
+                                                      0, loss, ra::WsGate{nullptr, 0, 0}, nullptr,
+                                                      0, 0u);
+  }
+  return launch_status();
+}
+
+// ---------------------------------------------------------------------------------------
 // Scratch for rope_attn_step_noalloc: lives in the library's device image, so every GPU that
 // loads the library holds it until exit.  Host code must not use the symbol's name as a device
 // address (it names a host-side shadow); the device address comes from cudaGetSymbolAddress.
@@ -909,6 +1114,30 @@ ra_status rope_attn_step_noalloc(const ra_problem* p, void* O, float* lse, float
   s = tc_fwd(p, O, lse, loss, ws, st);
   if (s != RA_OK) return s;
   return tc_bwd(p, O, lse, loss, dWQ, dWK, dWV, ws, 1, st);
+}
+
+size_t rope_attn_approx_workspace_bytes(const ra_problem* p) {
+  if (check_problem(p) != RA_OK) return 0;
+  return make_approx_layout(p).total;
+}
+
+ra_status rope_attn_approx_step(const ra_problem* p, void* O, float* loss, float* dWQ, float* dWK,
+                                float* dWV, void* ws, size_t ws_bytes, void* stream) {
+  ra_status s = check_problem(p);
+  if (s != RA_OK) return s;
+  if (!p->E || !O || !dWQ || !dWK || !dWV) return RA_ERR_INVALID_ARG;
+  if (!is_aligned(O, 16) || (loss && !is_aligned(loss, 4)) || !is_aligned(dWQ, 16) ||
+      !is_aligned(dWK, 16) || !is_aligned(dWV, 16))
+    return RA_ERR_ALIGNMENT;
+  if (!ws) return RA_ERR_WORKSPACE;
+  if (!is_aligned(ws, kAlignWs)) return RA_ERR_ALIGNMENT;
+  if (ws_bytes < make_approx_layout(p).total) return RA_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (p->dtype == RA_F32)
+    return p->d == 128 ? approx_step<float, 128>(p, O, loss, dWQ, dWK, dWV, ws, st)
+                       : approx_step<float, 64>(p, O, loss, dWQ, dWK, dWV, ws, st);
+  return p->d == 128 ? approx_step<__nv_bfloat16, 128>(p, O, loss, dWQ, dWK, dWV, ws, st)
+                     : approx_step<__nv_bfloat16, 64>(p, O, loss, dWQ, dWK, dWV, ws, st);
 }
 
 ra_status rope_attn_last_error(void* stream) {

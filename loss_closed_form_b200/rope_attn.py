@@ -22,7 +22,7 @@ EXPORTED = ("rope_attn_workspace_bytes", "rope_attn_fwd", "rope_attn_loss_bwd",
             "rope_attn_last_error", "rope_attn_status_string", "rope_attn_launch_count",
             "rope_attn_profile_enable", "rope_attn_profile_read", "rope_attn_kernel_name",
             "rope_attn_step_noalloc", "rope_attn_loss_bwd_inputs", "rope_attn_combined_weights",
-            "rope_attn_combined_grad")
+            "rope_attn_combined_grad", "rope_attn_approx_workspace_bytes", "rope_attn_approx_step")
 
 # Capacity of the static scratch behind rope_attn_step_noalloc (RA_NOALLOC_SCRATCH_BYTES).
 NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
@@ -86,6 +86,10 @@ def load() -> ctypes.CDLL:
     lib.rope_attn_combined_weights.argtypes = [vp, i32, i32, i32, vp, vp, vp]
     lib.rope_attn_combined_weights.restype = ctypes.c_int
     lib.rope_attn_combined_grad.argtypes = [vp, i32, i32, vp, vp]
+    lib.rope_attn_approx_workspace_bytes.argtypes = [P]
+    lib.rope_attn_approx_workspace_bytes.restype = sz
+    lib.rope_attn_approx_step.argtypes = [P, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.rope_attn_approx_step.restype = ctypes.c_int
     lib.rope_attn_combined_grad.restype = ctypes.c_int
     _lib = lib
     return lib
@@ -198,6 +202,20 @@ def step_noalloc(prob: Problem, O, lse, loss, dWQ, dWK, dWV, stream=None) -> Non
                                        _ptr(dWQ), _ptr(dWK), _ptr(dWV), _stream(stream))
     if st != RA_OK:
         raise RopeAttnError(st, "rope_attn_step_noalloc")
+
+
+def approx_workspace_bytes(prob: Problem) -> int:
+    return int(load().rope_attn_approx_workspace_bytes(ctypes.byref(prob)))
+
+
+def approx_step(prob: Problem, O, loss, dWQ, dWK, dWV, ws, stream=None) -> None:
+    """rope_attn_approx_step: the near-linear approximate method (degree-1 polynomial, low-rank
+    states): O, the loss and the approximate weight gradients."""
+    st = load().rope_attn_approx_step(ctypes.byref(prob), _ptr(O), _ptr(loss), _ptr(dWQ),
+                                      _ptr(dWK), _ptr(dWV), _ptr(ws),
+                                      ws.numel() * ws.element_size(), _stream(stream))
+    if st != RA_OK:
+        raise RopeAttnError(st, "rope_attn_approx_step")
 
 
 def last_error(stream=None) -> int:

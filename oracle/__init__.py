@@ -23,5 +23,9 @@ from .rope_attention import (  # noqa: F401
     rotation_matrix,
     combined_weight_literal,
     combined_weight_forward_backward,
+    poly_exp,
+    poly_features,
+    approx_instance_forward_backward,
+    approx_forward_backward,
     ORACLE_PARITY_PINNED,
 )

@@ -315,3 +315,113 @@ def combined_weight_forward_backward(inp: Dict[str, np.ndarray], causal: bool, b
     r = forward_backward(gen, causal, base)
     return {"loss": r["loss"], "O": r["O"], "lse": r["lse"],
             "dX": np.transpose(r["dWK"], (0, 2, 1)), "dWV": r["dWV"]}
+
+
+# ---------------------------------------------------------------------------------------
+# The near-linear approximate backward: polynomial method + low rank
+# ---------------------------------------------------------------------------------------
+# "RoPE Attention kan bijna lineair worden getraind", Methodologie 2 (Low-Rank
+# Benaderingsstrategie) and Resultaten (Theorem 5.7): under bounded entries the normalised
+# softmax s(x) is approximated by low-rank factors U1 V1^T built with a polynomial method, the
+# error term l(x) and beta(x) follow from it, gamma_1 = diag(s) beta is combined from the
+# factors of s and beta with row-wise Kronecker products, and gamma_2 = s s^T beta from
+# precomputed intermediates.  The pages name no degree, rank or construction.  Reading taken
+# here: exp(z) on the bounded scores z is replaced by its degree-g Taylor polynomial
+# P_g(z) = sum_{r <= g} z^r / r!, which factors exactly as P_g(q~_i . k~_j / sqrt(d)) =
+# phi(q~_i) . phi(k~_j) with the tensor-power features of ``poly_features``; s~ is P_g(Z)
+# normalised per row, and the gradient is the closed form with s~ in place of s:
+# l = s~ V - E, beta = l V^T, gamma = s~ o (beta - rowsum(s~ o beta)), dQ~ = gamma K~ / sqrt(d),
+# dK~ = gamma^T Q~ / sqrt(d), dV = s~^T l.  This is not the gradient of a loss built from s~
+# (d s~ / dz is not softmax-shaped); it is the page's approximation of each term of the exact
+# gradient.  The functions below evaluate that definition directly (quadratic in n) and give
+# the low-rank factors; the near-linear evaluation order is the CUDA path's.
+
+
+def poly_exp(z: np.ndarray, degree: int) -> np.ndarray:
+    """P_g(z) = sum_{r=0}^{g} z^r / r!, the truncated Taylor series of exp."""
+    z = np.asarray(z, F64)
+    out = np.zeros_like(z)
+    term = np.ones_like(z)
+    for r in range(degree + 1):
+        if r > 0:
+            term = term * z / r
+        out = out + term
+    return out
+
+
+def poly_features(X: np.ndarray, degree: int) -> np.ndarray:
+    """Rows phi(x) with phi(q) . phi(k) = P_g(q . k / sqrt(d)): the tensor powers x^(x)r of
+    every degree r <= g, each scaled by d^(-r/4) / sqrt(r!), side by side ([n][sum_r d^r])."""
+    X = np.asarray(X, F64)
+    n, d = X.shape
+    parts = [np.ones((n, 1), F64)]
+    cur = np.ones((n, 1), F64)
+    for r in range(1, degree + 1):
+        cur = np.einsum("ni,nj->nij", cur, X).reshape(n, -1)
+        parts.append(cur * (d ** (-r / 4.0)) / math.sqrt(math.factorial(r)))
+    return np.concatenate(parts, axis=1)
+
+
+def approx_instance_forward_backward(A1, A2, A3, E, WQ, WK, WV, pos, causal: bool, base: float,
+                                     degree: int, rb: int = 256) -> Dict[str, np.ndarray]:
+    """One instance with the polynomial-kernel softmax s~ = P_g(Z) / rowsum (masked entries 0):
+    O, the normaliser D, loss and the approximate gradient (see the section comment)."""
+    n, d = np.shape(A1)
+    c = 1.0 / math.sqrt(d)
+    Qt, Kt, V, phi = _project(A1, A2, A3, WQ, WK, WV, pos, base)
+    E = np.asarray(E, F64)
+    O = np.empty((n, d), F64)
+    Dn = np.empty(n, F64)
+    dQt = np.empty((n, d), F64)
+    dKt = np.zeros((n, d), F64)
+    dV = np.zeros((n, d), F64)
+    loss = 0.0
+    for r0 in range(0, n, rb):
+        r1 = min(n, r0 + rb)
+        rows = np.arange(r0, r1)
+        kend = r1 if causal else n
+        Z = (Qt[rows] @ Kt[:kend].T) * c
+        Pz = poly_exp(Z, degree)
+        if causal:
+            Pz = np.where(np.arange(kend)[None, :] > rows[:, None], 0.0, Pz)
+        Dn[r0:r1] = np.sum(Pz, axis=1)
+        s = Pz / Dn[r0:r1, None]                         # s~ (polynomial kernel, normalised)
+        O[r0:r1] = s @ V[:kend]
+        ell = O[r0:r1] - E[r0:r1]
+        loss += 0.5 * float(np.sum(ell * ell))
+        beta = ell @ V[:kend].T
+        gamma = gamma_closed_form(s, beta)               # gamma_1 - gamma_2 with s~
+        dQt[r0:r1] = (gamma @ Kt[:kend]) * c
+        dKt[:kend] += (gamma.T @ Qt[r0:r1]) * c
+        dV[:kend] += s.T @ ell
+    dQ = rope_rotate(dQt, -phi)
+    dK = rope_rotate(dKt, -phi)
+    A1, A2, A3 = (np.asarray(a, F64) for a in (A1, A2, A3))
+    return {"O": O, "D": Dn, "loss": loss, "dQt": dQt, "dKt": dKt, "dV": dV,
+            "dWQ": A1.T @ dQ, "dWK": A2.T @ dK, "dWV": A3.T @ dV}
+
+
+def approx_forward_backward(inp: Dict[str, np.ndarray], causal: bool, base: float, degree: int,
+                            heads: Optional[Iterable[int]] = None) -> Dict[str, np.ndarray]:
+    """All (b, h) instances (or those of ``heads``) of the approximate method: O, D, loss and
+    dWQ, dWK, dWV summed over the batch (entries of heads not computed are NaN)."""
+    B, H, n, d = inp["A1"].shape
+    O = np.full((B, H, n, d), np.nan)
+    Dn = np.full((B, H, n), np.nan)
+    dW = {k: np.full((H, d, d), np.nan) for k in ("dWQ", "dWK", "dWV")}
+    loss = 0.0
+    for h in _heads(inp, heads):
+        for k in dW:
+            dW[k][h] = 0.0
+        for b in range(B):
+            r = approx_instance_forward_backward(inp["A1"][b, h], inp["A2"][b, h],
+                                                 inp["A3"][b, h], inp["E"][b, h], inp["WQ"][h],
+                                                 inp["WK"][h], inp["WV"][h], inp["pos"], causal,
+                                                 base, degree)
+            O[b, h], Dn[b, h] = r["O"], r["D"]
+            loss += r["loss"]
+            for k in dW:
+                dW[k][h] += r[k]
+    out = {"O": O, "D": Dn, "loss": loss}
+    out.update(dW)
+    return out
