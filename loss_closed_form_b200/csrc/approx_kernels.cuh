@@ -21,8 +21,8 @@ namespace approx {
 constexpr int kChunk = 256;   // rows per state chunk
 constexpr int kThreads = 256;
 constexpr int kTile = 32;     // rows staged per step in the local-sum kernel
-constexpr int kRowBlk = 64;   // rows per apply CTA
-constexpr int kEBlk = 32;     // output columns per apply CTA
+constexpr int kRowBlk = 64;   // rows per apply CTA (8 per warp)
+constexpr int kEBlk = 64;     // output columns per apply CTA (2 per lane)
 
 // feature a (0 .. d) of the row x: 1 for a = 0, c4 * x[a - 1] otherwise (c4 = d^-1/4)
 __device__ __forceinline__ float feat(const float* __restrict__ x, int a, float c4) {
@@ -109,18 +109,33 @@ local_sum_kernel(const float* __restrict__ X, const float* __restrict__ x, const
 __global__ void state_scan_kernel(float* __restrict__ S, long long size, int nch, int mode) {
   const long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (e >= size) return;
+  constexpr int U = 8;  // chunks loaded before any is written: eight loads in flight per thread
+  float run = 0.f;
   if (mode == 2) {
-    float tot = 0.f;
-    for (int c = 0; c < nch; ++c) tot += S[(size_t)c * size + e];
-    for (int c = 0; c < nch; ++c) S[(size_t)c * size + e] = tot;
+    for (int c0 = 0; c0 < nch; c0 += U) {
+      float v[U];
+#pragma unroll
+      for (int k = 0; k < U; ++k) v[k] = c0 + k < nch ? S[(size_t)(c0 + k) * size + e] : 0.f;
+#pragma unroll
+      for (int k = 0; k < U; ++k) run += v[k];
+    }
+    for (int c = 0; c < nch; ++c) S[(size_t)c * size + e] = run;
     return;
   }
-  float run = 0.f;
-  for (int k = 0; k < nch; ++k) {
-    const int c = mode == 0 ? k : nch - 1 - k;
-    const float v = S[(size_t)c * size + e];
-    S[(size_t)c * size + e] = run;
-    run += v;
+  for (int k0 = 0; k0 < nch; k0 += U) {
+    float v[U];
+#pragma unroll
+    for (int k = 0; k < U; ++k) {
+      const int c = mode == 0 ? k0 + k : nch - 1 - (k0 + k);
+      v[k] = k0 + k < nch ? S[(size_t)c * size + e] : 0.f;
+    }
+#pragma unroll
+    for (int k = 0; k < U; ++k) {
+      if (k0 + k >= nch) break;
+      const int c = mode == 0 ? k0 + k : nch - 1 - (k0 + k);
+      S[(size_t)c * size + e] = run;
+      run += v[k];
+    }
   }
 }
 
@@ -128,71 +143,80 @@ __global__ void state_scan_kernel(float* __restrict__ S, long long size, int nch
 // Apply the states to rows r (of the chunk each row lies in):
 //   KRON:  out[r][e] += scale s_r sum_a f'_ra sum_b x'_rb S[a][b][e]
 //   !KRON: out[r][e] += scale s_r sum_a f'_ra S[a][e]
-// f'_ra = feat(X[r], a); s_r = ss[r] (or 1).  grid (ceil(n / 64), ceil(W / 32)), 256 threads:
-// warp w takes rows w, w + 8, ... of the block, its lane the output column.
+// f'_ra = feat(X[r], a); s_r = ss[r] (or 1).  grid (ceil(n / 64), ceil(W / 64)), 256 threads:
+// warp w takes rows 8 w .. 8 w + 7 of the block, its lane two output columns; the rows'
+// coefficients are stored transposed so that each step over u reads them with two broadcast
+// 16-byte loads and the state with one 8-byte load per lane (16 FMAs per three loads).
 // ---------------------------------------------------------------------------------------
 template <int D, bool KRON, int W>
 __global__ void __launch_bounds__(kThreads)
 apply_kernel(const float* __restrict__ X, const float* __restrict__ x, const float* __restrict__ ss,
              const float* __restrict__ S, float* __restrict__ out, int n, float c4, float scale) {
-  constexpr int NU = D + 1, LDU = NU + 1, LDX = D + 1;
-  extern __shared__ float sm[];
-  float* Xs = sm;                          // [64][D + 1] rows of X
-  float* xsm = Xs + kRowBlk * LDX;         // [64][NU + 1] rows of x (KRON)
-  float* St = xsm + (KRON ? kRowBlk * LDU : 0);  // KRON: [NU][32] of one a; else [NU][32]
+  constexpr int NU = D + 1;
+  extern __shared__ __align__(16) float sm[];
+  // [NU][64] per-row coefficients, transposed so that the 8 rows a warp handles are adjacent:
+  // fT[a][r] = f'_ra (the features), xT[b][r] = x'_rb (KRON)
+  float* fT = sm;
+  float* xT = fT + NU * kRowBlk;
+  float* St = xT + (KRON ? NU * kRowBlk : 0);   // [NU][64]: S[a][u][e0 ..] (KRON) or S[u][e0 ..]
   const int r0 = blockIdx.x * kRowBlk, e0 = blockIdx.y * kEBlk, tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
   const int nr = min(kRowBlk, n - r0);
   const int ch = r0 / kChunk;   // 64 divides kChunk: the block lies in one chunk
   const size_t state = (size_t)(KRON ? NU : 1) * NU * W;
   const float* Sc = S + ch * state;
-  for (int e = tid; e < kRowBlk * D; e += kThreads) {
-    const int rr = e / D, c = e - rr * D;
-    Xs[rr * LDX + c] = rr < nr ? X[(size_t)(r0 + rr) * D + c] : 0.f;
+  for (int e = tid; e < NU * kRowBlk; e += kThreads) {
+    const int a = e / kRowBlk, rr = e - a * kRowBlk;
+    fT[e] = rr < nr ? feat(X + (size_t)(r0 + rr) * D, a, c4) : 0.f;
+    if (KRON) xT[e] = rr < nr ? x[(size_t)(r0 + rr) * NU + a] : 0.f;
   }
-  if (KRON)
-    for (int e = tid; e < kRowBlk * NU; e += kThreads) {
-      const int rr = e / NU, c = e - rr * NU;
-      xsm[rr * LDU + c] = rr < nr ? x[(size_t)(r0 + rr) * NU + c] : 0.f;
-    }
-  const int ecol = e0 + lane;
-  float acc[8];
+  // warp w: rows 8 w .. 8 w + 7; lane: output columns e0 + 2 lane, e0 + 2 lane + 1
+  const int rb = 8 * warp;
+  float acc[8][2];
 #pragma unroll
-  for (int k = 0; k < 8; ++k) acc[k] = 0.f;
+  for (int k = 0; k < 8; ++k) acc[k][0] = acc[k][1] = 0.f;
   for (int a = 0; a < (KRON ? NU : 1); ++a) {
     __syncthreads();
-    // KRON: S[a][u][e0 ..], else S[u][e0 ..] (u runs over the features)
     const float* src = Sc + (KRON ? (size_t)a * NU * W : 0);
     for (int e = tid; e < NU * kEBlk; e += kThreads) {
       const int u = e / kEBlk, c = e - u * kEBlk;
       St[e] = (e0 + c < W) ? src[(size_t)u * W + e0 + c] : 0.f;
     }
     __syncthreads();
+    float dot[8][2];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) dot[k][0] = dot[k][1] = 0.f;
+    const float* cu = KRON ? xT : fT;   // KRON: sum over b of x'_rb S[a][b][e]; else over a
+    for (int u = 0; u < NU; ++u) {
+      const float4 c0 = *reinterpret_cast<const float4*>(cu + u * kRowBlk + rb);
+      const float4 c1 = *reinterpret_cast<const float4*>(cu + u * kRowBlk + rb + 4);
+      const float2 sv = *reinterpret_cast<const float2*>(St + u * kEBlk + 2 * lane);
+      const float cr[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        dot[k][0] = fmaf(cr[k], sv.x, dot[k][0]);
+        dot[k][1] = fmaf(cr[k], sv.y, dot[k][1]);
+      }
+    }
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
-      const int rr = warp + 8 * k;
-      const float* xr = Xs + rr * LDX;
-      if (KRON) {
-        const float* xv = xsm + rr * LDU;
-        float dot = 0.f;
-        for (int b = 0; b < NU; ++b) dot = fmaf(xv[b], St[b * kEBlk + lane], dot);
-        acc[k] = fmaf(feat(xr, a, c4), dot, acc[k]);
-      } else {
-        float dot = 0.f;
-        for (int u = 0; u < NU; ++u) dot = fmaf(feat(xr, u, c4), St[u * kEBlk + lane], dot);
-        acc[k] += dot;
-      }
+      const float fa = KRON ? fT[a * kRowBlk + rb + k] : 1.f;
+      acc[k][0] = fmaf(fa, dot[k][0], acc[k][0]);
+      acc[k][1] = fmaf(fa, dot[k][1], acc[k][1]);
     }
   }
-  if (ecol < W)
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const int rr = warp + 8 * k;
-      if (rr < nr) {
-        const int r = r0 + rr;
-        out[(size_t)r * W + ecol] += scale * (ss ? ss[r] : 1.f) * acc[k];
-      }
+  for (int k = 0; k < 8; ++k) {
+    const int rr = rb + k;
+    if (rr >= nr) continue;
+    const int r = r0 + rr;
+    const float sr = scale * (ss ? ss[r] : 1.f);
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      const int ecol = e0 + 2 * lane + q;
+      if (ecol < W) out[(size_t)r * W + ecol] += sr * acc[k][q];
     }
+  }
 }
 
 // ---------------------------------------------------------------------------------------

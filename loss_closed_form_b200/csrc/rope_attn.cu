@@ -818,7 +818,7 @@ void apx_apply(const float* X, const float* x, const float* ss, const float* S, 
                float scale, cudaStream_t st) {
   using namespace ra::approx;
   constexpr int NU = D + 1;
-  const size_t smem = (size_t)(kRowBlk * (D + 1) + (KRON ? kRowBlk * (NU + 1) : 0) + NU * kEBlk) * 4;
+  const size_t smem = (size_t)(NU * kRowBlk * (KRON ? 2 : 1) + NU * kEBlk) * 4;
   auto k = apply_kernel<D, KRON, W>;
   cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   Launch l(K_APX_APPLY, st);
