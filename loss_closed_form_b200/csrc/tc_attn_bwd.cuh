@@ -430,7 +430,9 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         tma_store_3d(&tm_dv, sbase + C::Q_OFF + C::KTILE + b * C::KBLK, 64 * b, kt * C::BK, bh);
       }
       bulk_commit();
-      bulk_wait0();  // the stores have landed before the CTA leaves
+      // the stores have read the staging before the CTA leaves (their writes complete with
+      // the kernel)
+      bulk_wait_read0();
     }
   } else {
     // ------------------------------------------------------------------ dQ~ drain (warps 8-11)
@@ -477,7 +479,7 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       }
       if (!__all_sync(0xffffffffu, iok)) break;  // leave the loop together
     }
-    if (issuer) bulk_wait0();  // the reductions have landed before the CTA leaves
+    if (issuer) bulk_wait_read0();  // the reductions have read the staging tile
   }
   tc_fence_before();
   __syncthreads();

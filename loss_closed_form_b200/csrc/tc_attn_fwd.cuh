@@ -496,7 +496,9 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
         bulk_commit();
       }
     }
-    if (ok && r == 0) bulk_wait0();  // the stores have landed before the CTA leaves
+    // the stores have read the staging before the CTA leaves (their writes complete with the
+    // kernel)
+    if (ok && r == 0) bulk_wait_read0();
     // per-warp partial of 1/2 sum l^2 (fixed order: deterministic)
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);

@@ -53,6 +53,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Same test, but a thread whose phase has not completed is suspended until it does or about
+// `ns` nanoseconds have passed: a waiting warp takes no issue slots from the warps it shares
+// its sub-partition with.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity, uint32_t ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(ns)
+      : "memory");
+  return ok != 0;
+}
+
 // The CTA's abort flag lives in shared memory and is read / written with explicit
 // shared-space accesses (a generic pointer would send every poll through L1TEX).
 __device__ __forceinline__ int abort_get(uint32_t flag) {
@@ -64,6 +79,10 @@ __device__ __forceinline__ void abort_set(uint32_t flag, int v) {
   asm volatile("st.volatile.shared.s32 [%0], %1;" ::"r"(flag), "r"(v) : "memory");
 }
 
+// Longest suspension of one try_wait inside the bounded waits (the abort flag and the time
+// limit are checked between two of them).
+constexpr uint32_t kWaitSleepNs = 10000;
+
 // Wait for the phase with parity `parity` of barrier `bar` to complete.  Gives up when the
 // CTA's abort flag (shared address `abort_flag`) is set, or after `limit_ns` of global time:
 // then records a timeout in the library status word, sets the abort flag and returns false.
@@ -72,7 +91,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint32_
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait_sleep(bar, parity, kWaitSleepNs)) return true;
     if (abort_get(abort_flag)) return false;
     if (globaltimer() - t0 > limit_ns) {
       flag_error(kDevTimeout);
