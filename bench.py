@@ -51,6 +51,8 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-input-grads", action="store_true")
+    ap.add_argument("--deterministic", action="store_true",
+                    help="the backward's fixed-order (bitwise repeatable) mode")
     ap.add_argument("--approx", action="store_true",
                     help="also time the near-linear approximate method (rope_attn_approx_step)")
     return ap.parse_args()
@@ -177,8 +179,9 @@ def run_ours(args, rank, world, local_rank):
     host["pos"] = torch.from_numpy(inp["pos"]).pin_memory()
     del inp
     t = {k: v.to(dev) for k, v in host.items()}
+    det = bool(getattr(args, "deterministic", False))
     m = ra.RopeAttention(t["A1"], t["A2"], t["A3"], t["WQ"], t["WK"], t["WV"], t["E"],
-                         t["pos"], w.causal, w.rope_base)
+                         t["pos"], w.causal, w.rope_base, deterministic=det)
     stream = torch.cuda.current_stream(dev)
     flops = flop_count(w)
 
@@ -228,7 +231,7 @@ def run_ours(args, rank, world, local_rank):
         slots = [(t, m)]
         t2 = {k: torch.empty_like(v) for k, v in t.items()}
         m2 = ra.RopeAttention(t2["A1"], t2["A2"], t2["A3"], t2["WQ"], t2["WK"], t2["WV"],
-                              t2["E"], t2["pos"], w.causal, w.rope_base)
+                              t2["E"], t2["pos"], w.causal, w.rope_base, deterministic=det)
         slots.append((t2, m2))
         out_host = [{"loss": torch.empty((), dtype=torch.float32).pin_memory(),
                      "dWQ": torch.empty_like(m.dWQ, device="cpu").pin_memory(),
@@ -357,7 +360,7 @@ def run_ours(args, rank, world, local_rank):
         "steps": args.steps, "warmup": max(3, args.warmup),
         "ms_per_step": round(ms_max / args.steps, 4), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
-        "config": workload_config(w, world),
+        "config": dict(workload_config(w, world), **({"deterministic": True} if det else {})),
         "frac_of_bf16_peak": round(value / world / pk["bf16_tflops"], 4),
         "tokens_per_s": round(world * w.B * w.n * args.steps / (ms_max * 1e-3), 1),
         "roofline": roof,

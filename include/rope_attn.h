@@ -73,6 +73,11 @@ typedef struct {
   const void* WK;          /* device [H][d][d]                                            */
   const void* WV;          /* device [H][d][d]                                            */
   const void* E;           /* device [B][H][n][d]: target; may be NULL in rope_attn_fwd   */
+  int32_t deterministic;   /* 0 or 1.  1: the backward adds the per-key-tile parts of the  */
+                           /* query-side gradient in a fixed order, so dWQ, dWK, dWV and   */
+                           /* dA1..dA3 are bitwise the same on every run (a little slower); */
+                           /* 0: in whatever order the key tiles finish.  Exact path only;  */
+                           /* not part of the workspace tag                                 */
 } ra_problem;
 
 /*

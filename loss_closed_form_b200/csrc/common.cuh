@@ -30,6 +30,39 @@ enum DeviceStatus : int {
 
 __device__ __forceinline__ void flag_error(int code) { atomicMax(&g_status, code); }
 
+// ---- ordered accumulation (the backward's deterministic mode) ------------------------------
+// A counter per accumulator tile says whose turn it is: contributor k adds its part once the
+// counter reads k and passes the turn on afterwards, so the fp32 sums run in the order
+// 0, 1, 2, ... on every run.  Contributors with a lower index are launched earlier (they are
+// CTAs of lower linear index in the same grid), so each wait ends; it is bounded all the same.
+
+// Wait (bounded by limit_ns of global time) until *turn == want; false after a timeout, which
+// is also recorded in the status word.
+__device__ __forceinline__ bool turn_wait(const unsigned* turn, unsigned want,
+                                          unsigned long long limit_ns) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(turn) : "memory");
+  if (v == want) return true;
+  unsigned long long t0, t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t0));
+  while (true) {
+    __nanosleep(64);
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(turn) : "memory");
+    if (v == want) return true;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    if (t - t0 > limit_ns) {
+      flag_error(kDevTimeout);
+      return false;
+    }
+  }
+}
+
+// Pass the turn on: everything this thread wrote (or saw written by the threads it
+// synchronised with) before is visible to the next contributor.
+__device__ __forceinline__ void turn_pass(unsigned* turn) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(turn) : "memory");
+}
+
 // Header at the start of every workspace: which problem's intermediates the workspace holds.
 // The last kernel of a forward or backward call writes it; the backward's recomputation kernels
 // read it on the device and skip their work when it already holds what they would write.

@@ -127,6 +127,7 @@ struct Layout {
   size_t dv16;       // bf16 [B][H][n][d] (bf16 path)
   size_t dw_part;    // float [3][H][nsplit][d][d]
   size_t loss_part;  // double [nparts]
+  size_t turn;       // unsigned [B][H][turn_stride]: turn counters of the deterministic mode
   size_t total;
   int inter;         // bytes per intermediate element
   int nsplit;        // weight-gradient row splits per head
@@ -134,6 +135,7 @@ struct Layout {
   int nparts;        // capacity of the loss partial sums
   int nparts_fwd;    // partial sums the forward writes
   int nparts_pre;    // partial sums the backward's own l = O - E pass writes
+  int turn_stride;   // turn counters per instance: one per 32-row query tile
 };
 
 bool is_aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
@@ -143,6 +145,7 @@ ra_status check_problem(const ra_problem* p) {
   if (p->B < 1 || p->H < 1 || p->n < 1 || p->d < 1) return RA_ERR_INVALID_ARG;
   if (p->dtype != RA_F32 && p->dtype != RA_BF16) return RA_ERR_INVALID_ARG;
   if (p->causal != 0 && p->causal != 1) return RA_ERR_INVALID_ARG;
+  if (p->deterministic != 0 && p->deterministic != 1) return RA_ERR_INVALID_ARG;
   if (!(p->rope_base > 0.0) || !isfinite(p->rope_base)) return RA_ERR_INVALID_ARG;
   if (!p->A1 || !p->A2 || !p->A3 || !p->WQ || !p->WK || !p->WV) return RA_ERR_INVALID_ARG;
   if (p->d != 64 && p->d != 128) return RA_ERR_UNSUPPORTED;
@@ -230,6 +233,8 @@ Layout make_layout(const ra_problem* p) {
   L.dv16 = take(tcp ? act * 2 : 0);
   L.dw_part = take(3 * H * (size_t)L.nsplit * d * d * sizeof(float));
   L.loss_part = take((size_t)L.nparts * sizeof(double));
+  L.turn_stride = (int)((n + 31) / 32);
+  L.turn = take(B * H * (size_t)L.turn_stride * sizeof(unsigned));
   L.total = off;
   return L;
 }
@@ -391,7 +396,8 @@ void bwd_prep(const ra_problem* p, const Layout& L, const void* O, void* ws, con
                                      ra::simt::kThreads, 0, st>>>(
       (const T*)O, (const T*)p->E, at<TL>(ws, L.ell), at<float>(ws, L.delta),
       at<double>(ws, L.loss_part), p->n, p->d, (int)BH, at<float2>(ws, L.rope), p->pos,
-      p->rope_base, at<float4>(ws, L.dqt), BH * p->n * p->d / 4, g.recompute, g.zero);
+      p->rope_base, at<float4>(ws, L.dqt), BH * p->n * p->d / 4, g.recompute, g.zero,
+      p->deterministic ? at<unsigned>(ws, L.turn) : nullptr, BH * L.turn_stride);
 }
 
 // ---------------------------------------------------------------------------------------
@@ -658,6 +664,8 @@ ra_status tc_bwd_launch(const ra_problem* p, const Layout& L, const float* lse, 
   BwdParams bp;
   bp.lse = lse;
   bp.delta = at<float>(ws, L.delta);
+  bp.turn = p->deterministic ? at<unsigned>(ws, L.turn) : nullptr;
+  bp.turn_stride = L.turn_stride;
   bp.n = n;
   bp.BH = BH;
   bp.nk = (n + C::BK - 1) / C::BK;
@@ -696,7 +704,8 @@ ra_status simt_bwd(const ra_problem* p, const void* O, const float* lse, float* 
     attn_bwd_kernel<float><<<grid, kThreads, smem, st>>>(
         at<float>(ws, L.qt), at<float>(ws, L.kt), at<float>(ws, L.v), at<float>(ws, L.ell), lse,
         at<float>(ws, L.delta), at<float>(ws, L.dqt), at<float>(ws, L.dkt), at<float>(ws, L.dv),
-        n, d, p->causal, scale, scale * ra::kLog2e);
+        n, d, p->causal, scale, scale * ra::kLog2e,
+        p->deterministic ? at<unsigned>(ws, L.turn) : nullptr, L.turn_stride, wait_limit_ns());
   }
   {
     size_t smem = (size_t)2 * 16 * d * sizeof(float);

@@ -265,7 +265,8 @@ __global__ void __launch_bounds__(kThreads)
 bwd_prep_kernel(const T* __restrict__ O, const T* __restrict__ E, TL* __restrict__ ell,
                 float* __restrict__ delta, double* __restrict__ loss_part, int n, int d, int BH,
                 float2* __restrict__ tab, const int32_t* __restrict__ pos, double base,
-                float4* __restrict__ dq, long long n4, WsGate recompute, WsGate zero) {
+                float4* __restrict__ dq, long long n4, WsGate recompute, WsGate zero,
+                unsigned* __restrict__ turn, long long nturn) {
   __shared__ double red[kThreads / 32];
   const bool rec = !gate_skip(recompute), zer = !gate_skip(zero);
   if (rec) {
@@ -280,12 +281,18 @@ bwd_prep_kernel(const T* __restrict__ O, const T* __restrict__ E, TL* __restrict
     for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n4;
          i += (long long)gridDim.x * blockDim.x)
       dq[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+  // the deterministic mode's turn counters (not gated: every backward starts them at zero)
+  if (turn)
+    for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < nturn;
+         i += (long long)gridDim.x * blockDim.x)
+      turn[i] = 0u;
 }
 
 // ---------------------------------------------------------------------------------------
 // Backward over one key tile of 32 rows, looping over query tiles of 32:
 //   P^T = exp(S^T - lse), beta^T = V l^T, gamma^T = P^T o (beta^T - delta)
-//   dV += P^T l,  dK~ += gamma^T Q~ / sqrt(d),  dQ~ += gamma K~ / sqrt(d) (atomic adds)
+//   dV += P^T l,  dK~ += gamma^T Q~ / sqrt(d),  dQ~ += gamma K~ / sqrt(d) (atomic adds, or
+//   with `turn` in the fixed key-tile order of the deterministic mode)
 // grid (ceil(n/32), B*H), 256 threads, thread (r = tid/8, g = tid%8).
 // ---------------------------------------------------------------------------------------
 template <class TX>
@@ -294,7 +301,8 @@ attn_bwd_kernel(const TX* __restrict__ Qt, const TX* __restrict__ Kt,
                 const TX* __restrict__ V, const TX* __restrict__ ell,
                 const float* __restrict__ lse, const float* __restrict__ delta,
                 float* __restrict__ dQt, float* __restrict__ dKt, float* __restrict__ dV,
-                int n, int d, int causal, float scale, float scale_log2) {
+                int n, int d, int causal, float scale, float scale_log2, unsigned* turn,
+                int turn_stride, unsigned long long limit_ns) {
   extern __shared__ float smem[];
   const int ld = d + 4;
   float* Ks = smem;
@@ -305,7 +313,10 @@ attn_bwd_kernel(const TX* __restrict__ Qt, const TX* __restrict__ Kt,
   float* GT = PT + kRows * 33;   // [32][33]
   float* lse_s = GT + kRows * 33;
   float* del_s = lse_s + kRows;
-  const int bh = blockIdx.y, j0 = blockIdx.x * kRows, tid = threadIdx.x;
+  // deterministic mode: key tiles in reverse order (the shortest first when causal), each
+  // taking its turn on a query tile after the higher key tiles that share it
+  const int kt = turn ? static_cast<int>(gridDim.x - 1 - blockIdx.x) : static_cast<int>(blockIdx.x);
+  const int bh = blockIdx.y, j0 = kt * kRows, tid = threadIdx.x;
   const int r = tid >> 3, g = tid & 7;
   const int key = j0 + r;
   const size_t base = (size_t)bh * n * d;
@@ -361,17 +372,36 @@ attn_bwd_kernel(const TX* __restrict__ Qt, const TX* __restrict__ Kt,
     }
     // dQ~ rows of this query tile: thread (r -> query row, g -> columns)
     const int qrow = i0 + r;
-    if (qrow < n) {
-      float aq[16];
+    float aq[16];
 #pragma unroll
-      for (int u = 0; u < 16; ++u) aq[u] = 0.f;
+    for (int u = 0; u < 16; ++u) aq[u] = 0.f;
+    if (qrow < n) {
       for (int k = 0; k < kRows; ++k) {
         const float gm = GT[k * 33 + r];
 #pragma unroll
         for (int u = 0; u < 16; ++u)
           if (u < ncol) aq[u] = fmaf(gm, Ks[k * ld + g + 8 * u], aq[u]);
       }
-      float* dst = dQt + base + (size_t)qrow * d;
+    }
+    float* dst = dQt + base + (size_t)qrow * d;
+    if (turn) {
+      // deterministic mode: query tile qt gets the parts of key tiles kmax, kmax - 1, ..., 0
+      // in that order (all of them contribute to it), so this one adds its part once
+      // kmax - kt others have (read-modify-write through L2)
+      const int qt = i0 / kRows, nkt = static_cast<int>(gridDim.x);
+      const int kmax = causal ? min(nkt - 1, qt) : nkt - 1;
+      unsigned* tc = turn + (size_t)bh * turn_stride + qt;
+      if (tid == 0) turn_wait(tc, static_cast<unsigned>(kmax - kt), limit_ns);
+      __syncthreads();
+      if (qrow < n) {
+#pragma unroll
+        for (int u = 0; u < 16; ++u)
+          if (u < ncol) __stcg(dst + g + 8 * u, __ldcg(dst + g + 8 * u) + aq[u] * scale);
+      }
+      __threadfence();
+      __syncthreads();
+      if (tid == 0) turn_pass(tc);
+    } else if (qrow < n) {
 #pragma unroll
       for (int u = 0; u < 16; ++u)
         if (u < ncol) atomicAdd(dst + g + 8 * u, aq[u] * scale);

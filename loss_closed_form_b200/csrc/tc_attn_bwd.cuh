@@ -74,6 +74,8 @@ struct BwdCfg {
   static_assert(TABT <= 2 * KTILE && 2 * KTILE <= 2 * NSQ * QTILE, "epilogue staging");
   static constexpr int THREADS = 448;
   static constexpr int W_DRAIN = 8, W_PROD = 12, W_MMA = 13;
+  // deterministic mode: steps between a query tile's reduction and passing its turn on
+  static constexpr int TURN_LAG = 1;
   // TMEM columns: step buffer b at 128 b holds S^T (columns 0-63) and beta^T (64-127); the
   // softmax warpgroup h then writes P^T at 32 h and gamma^T at 32 h + 16 (16 columns each, two
   // bf16 per column) and dQ~^T is accumulated at 64
@@ -86,6 +88,10 @@ struct BwdCfg {
 struct BwdParams {
   const float* lse;     // [BH][n]
   const float* delta;   // [BH][n]
+  // deterministic mode: [BH][turn_stride] turn counters, one per 64-row query tile, zero at
+  // launch (null: the dQ~ tiles are added in whatever order the key tiles get there)
+  unsigned* turn;
+  int turn_stride;
   int n, BH, nk, causal;
   int hgroup;          // heads per scheduling group (their Q~, l, dQ~ fit in L2 together)
   float scale;         // 1 / sqrt(d)
@@ -129,7 +135,9 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
   // group of p.hgroup heads, whose Q~, l and dQ~ stay in L2 together, runs its longest key
   // tiles first (key tile 0 sees the most query tiles when causal) across all of its heads
   // and the grid ends on short CTAs
-  const int kt = blockIdx.y;
+  // deterministic mode: the shortest key tiles (highest index when causal) are dispatched
+  // first, and take their turn first on every query tile (see the drain)
+  const int kt = p.turn ? p.nk - 1 - static_cast<int>(blockIdx.y) : static_cast<int>(blockIdx.y);
   const int bh = blockIdx.z * gridDim.x + blockIdx.x;  // gridDim.x = p.hgroup
   if (bh >= p.BH) return;  // the last group may hold fewer heads
   const int n = p.n;
@@ -444,6 +452,7 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     const bool has_row = (D == 128) || lane < 16;
     const uint32_t stage = sbase + C::DQS_OFF;
     const bool issuer = tid == 32 * C::W_DRAIN;
+    int passed = 0;  // query tiles whose turn this key tile has passed on (deterministic mode)
     for (int ii = 0; ii < NI; ++ii) {
       const int b = ii & 1;
       if (!mbar_wait_warp(b_dqfull(b), (ii >> 1) & 1, abort_flag, lim)) break;
@@ -470,7 +479,34 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       bool iok = true;
       if (issuer) {
         iok = mbar_wait(b_dqsfull, ii & 1, abort_flag, lim);
-        if (iok) {
+        if (iok && p.turn) {
+          // deterministic mode: query tile q gets the parts of key tiles kmax(q), kmax(q) - 1,
+          // ..., 0 in that order (all of them contribute to it), so key tile kt adds its part
+          // once kmax(q) - kt others have.  Those others were dispatched before this CTA and
+          // reach q two query tiles sooner.  The turn of a tile passes on once its reduction
+          // has landed, checked TURN_LAG steps later (when at most the TURN_LAG newer ones are
+          // in flight: the key tile after this one in the order reaches q later still).
+          const int q = i_start + ii;
+          const int kmax = p.causal ? min(p.nk - 1, (q * C::BQ + C::BQ - 1) / C::BK) : p.nk - 1;
+          unsigned* tc = p.turn + (size_t)bh * p.turn_stride + q;
+          if (turn_wait(tc, static_cast<unsigned>(kmax - kt), lim)) {
+            fence_proxy_async_global();
+            tma_reduce_add_3d(&tm_dq, stage, 0, (i_start + ii) * C::BQ, bh);
+            bulk_commit();
+            bulk_wait_read0();
+            mbar_arrive(b_dqsfree);
+            if (passed <= ii - C::TURN_LAG) {
+              bulk_wait_n<C::TURN_LAG>();
+              fence_proxy_async_global();
+              turn_pass(tc - (ii - passed));
+              ++passed;
+            }
+          } else {
+            abort_set(abort_flag, 1);  // given up: the turns still pass, the status says so
+            iok = false;
+            mbar_arrive(b_dqsfree);
+          }
+        } else if (iok) {
           tma_reduce_add_3d(&tm_dq, stage, 0, (i_start + ii) * C::BQ, bh);
           bulk_commit();
           bulk_wait_read0();
@@ -480,6 +516,14 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       if (!__all_sync(0xffffffffu, iok)) break;  // leave the loop together
     }
     if (issuer) bulk_wait_read0();  // the reductions have read the staging tile
+    if (issuer && p.turn) {
+      // the last tile's reduction has landed; after an abort, the query tiles this key tile
+      // has not added to pass their turn all the same, so the key tiles after it do not wait
+      // out their limit
+      bulk_wait0();
+      fence_proxy_async_global();
+      for (int q = passed; q < NI; ++q) turn_pass(p.turn + (size_t)bh * p.turn_stride + i_start + q);
+    }
   }
   tc_fence_before();
   __syncthreads();

@@ -385,21 +385,27 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
           }
         }
       }
-      float ps0 = 0.f, ps1 = 0.f;
+      // exponent arguments and row sums two columns per packed FFMA / FADD
+      const uint64_t sc2 = f32x2(p.scale_log2, p.scale_log2), nm2 = f32x2(-m, -m);
+      uint64_t ps2a = f32x2(0.f, 0.f), ps2b = f32x2(0.f, 0.f);
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          const float p0 = ex2(fmaf(x[32 * c + 2 * i], p.scale_log2, -m));
-          const float p1 = ex2(fmaf(x[32 * c + 2 * i + 1], p.scale_log2, -m));
-          ps0 += p0;
-          ps1 += p1;
+          const float2 y =
+              unpack_f32x2(ffma2(f32x2(x[32 * c + 2 * i], x[32 * c + 2 * i + 1]), sc2, nm2));
+          const float p0 = ex2(y.x), p1 = ex2(y.y);
+          if (i & 1)
+            ps2b = fadd2(ps2b, f32x2(p0, p1));
+          else
+            ps2a = fadd2(ps2a, f32x2(p0, p1));
           pk[i] = pack_bf16x2(p0, p1);
         }
         tmem_st16(p_col + 16 * c, pk);
       }
-      l += ps0 + ps1;
+      const float2 ps = unpack_f32x2(fadd2(ps2a, ps2b));
+      l += ps.x + ps.y;
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive_warp(b_pfull(t));

@@ -128,6 +128,11 @@ __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
+// Order this thread's global-memory accesses between the generic proxy (loads, stores,
+// atomics) and the async proxy (TMA bulk copies and reductions).
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
 
 // ---------------------------------------------------------------------------------------
 // TMA (no cluster multicast anywhere in this library)
@@ -442,6 +447,11 @@ __device__ __forceinline__ void bulk_wait_read0() {
 // Wait until every committed bulk group has completed.
 __device__ __forceinline__ void bulk_wait0() {
   asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+// Wait until at most the N most recently committed bulk groups are still in flight.
+template <int N>
+__device__ __forceinline__ void bulk_wait_n() {
+  asm volatile("cp.async.bulk.wait_group %0;" ::"n"(N) : "memory");
 }
 
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,

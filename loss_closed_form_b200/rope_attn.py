@@ -36,7 +36,7 @@ class Problem(ctypes.Structure):
         ("rope_base", ctypes.c_double), ("pos", ctypes.c_void_p),
         ("A1", ctypes.c_void_p), ("A2", ctypes.c_void_p), ("A3", ctypes.c_void_p),
         ("WQ", ctypes.c_void_p), ("WK", ctypes.c_void_p), ("WV", ctypes.c_void_p),
-        ("E", ctypes.c_void_p),
+        ("E", ctypes.c_void_p), ("deterministic", ctypes.c_int32),
     ]
 
 
@@ -117,10 +117,12 @@ def _stream(stream) -> Optional[int]:
 
 
 def make_problem(A1, A2, A3, WQ, WK, WV, E=None, pos=None, causal=False,
-                 rope_base=10000.0) -> Problem:
+                 rope_base=10000.0, deterministic=False) -> Problem:
     """Build an ``ra_problem`` from tensors (or raw device pointers with explicit shapes).
 
     A1, A2, A3, E: [B][H][n][d]; WQ, WK, WV: [H][d][d]; pos: [n] int32 or None.
+    deterministic: the backward adds its per-key-tile parts in a fixed order (bitwise
+    repeatable gradients).
     """
     import torch
     B, H, n, d = A1.shape
@@ -136,7 +138,8 @@ def make_problem(A1, A2, A3, WQ, WK, WV, E=None, pos=None, causal=False,
     if pos is not None and pos.dtype != torch.int32:
         raise TypeError("pos must be int32")
     return Problem(B, H, n, d, dt, int(bool(causal)), float(rope_base), _ptr(pos),
-                   _ptr(A1), _ptr(A2), _ptr(A3), _ptr(WQ), _ptr(WK), _ptr(WV), _ptr(E))
+                   _ptr(A1), _ptr(A2), _ptr(A3), _ptr(WQ), _ptr(WK), _ptr(WV), _ptr(E),
+                   int(bool(deterministic)))
 
 
 def workspace_bytes(prob: Problem) -> int:
@@ -261,10 +264,12 @@ class RopeAttention:
     forward's workspace, and returns (loss, dWQ, dWK, dWV) as device tensors.
     """
 
-    def __init__(self, A1, A2, A3, WQ, WK, WV, E, pos=None, causal=False, rope_base=10000.0):
+    def __init__(self, A1, A2, A3, WQ, WK, WV, E, pos=None, causal=False, rope_base=10000.0,
+                 deterministic=False):
         import torch
         self.inputs = (A1, A2, A3, WQ, WK, WV, E, pos)
-        self.prob = make_problem(A1, A2, A3, WQ, WK, WV, E, pos, causal, rope_base)
+        self.prob = make_problem(A1, A2, A3, WQ, WK, WV, E, pos, causal, rope_base,
+                                 deterministic)
         B, H, n, d = A1.shape
         dev = A1.device
         self.O = torch.empty_like(A1)

@@ -5,6 +5,8 @@
 //   descriptor form the library uses is checked in isolation against torch.
 // probe_timeout: a kernel waits on an mbarrier that nothing arrives on; the bounded wait
 //   must give up, record a timeout in the status word and return (no trap, no hang).
+// probe_turn: the turn counters of the ordered (deterministic) accumulation: CTAs take turns
+//   in a given order and log it, or one waits for a turn that never comes and gives up.
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -158,6 +160,17 @@ __global__ void probe_timeout_kernel(unsigned long long limit_ns, int* waited_ok
   if (threadIdx.x == 0) *waited_ok = ok ? 1 : 0;
 }
 
+// CTA b takes turn b (or gridDim.x - 1 - b) and writes its index at that position of `log`.
+__global__ void probe_turn_kernel(unsigned* counter, int* log, unsigned long long limit_ns,
+                                  int reverse, int* all_ok) {
+  if (threadIdx.x != 0) return;
+  const unsigned me = reverse ? gridDim.x - 1 - blockIdx.x : blockIdx.x;
+  if (!turn_wait(counter, me, limit_ns)) atomicExch(all_ok, 0);
+  if (me < gridDim.x) log[me] = static_cast<int>(blockIdx.x);
+  __threadfence();
+  turn_pass(counter);
+}
+
 __global__ void probe_exp2_kernel(const float* __restrict__ x, float* __restrict__ poly,
                                   float* __restrict__ ref, int n) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
@@ -187,6 +200,38 @@ int probe_mma(const void* A, const void* B, float* D, int M, int N, int K, int a
       (const __nv_bfloat16*)A, (const __nv_bfloat16*)B, D, M, N, K, a_mn, b_mn, a_tmem,
       2000000000ull);
   return (int)cudaGetLastError();
+}
+
+// nblocks CTAs take turns on a counter starting at `start` (CTA b waits for turn b, or
+// nblocks - 1 - b with reverse); log_host[k] gets the CTA that took turn k (nblocks ints),
+// *ok_host whether every wait succeeded, *final_host the counter at the end.  Returns the
+// status word (1 after a wait that gave up), or a negative value if a CUDA call failed.
+int probe_turn(int nblocks, int reverse, unsigned start, unsigned long long limit_ns,
+               int* log_host, int* ok_host, unsigned* final_host) {
+  if (nblocks < 1 || nblocks > 128) return -1;
+  unsigned* counter = nullptr;
+  int* log = nullptr;
+  int* ok = nullptr;
+  if (cudaMalloc(&counter, sizeof(unsigned)) != cudaSuccess) return -2;
+  if (cudaMalloc(&log, nblocks * sizeof(int)) != cudaSuccess) return -2;
+  if (cudaMalloc(&ok, sizeof(int)) != cudaSuccess) return -2;
+  const int one = 1, zero = 0;
+  cudaMemcpy(counter, &start, sizeof(unsigned), cudaMemcpyHostToDevice);
+  cudaMemset(log, 0xFF, nblocks * sizeof(int));
+  cudaMemcpy(ok, &one, sizeof(int), cudaMemcpyHostToDevice);
+  cudaMemcpyToSymbol(ra::g_status, &zero, sizeof(int));
+  probe_turn_kernel<<<nblocks, 32>>>(counter, log, limit_ns, reverse, ok);
+  if (cudaDeviceSynchronize() != cudaSuccess) return -3;
+  int st = 0;
+  cudaMemcpyFromSymbol(&st, ra::g_status, sizeof(int));
+  cudaMemcpy(log_host, log, nblocks * sizeof(int), cudaMemcpyDeviceToHost);
+  cudaMemcpy(ok_host, ok, sizeof(int), cudaMemcpyDeviceToHost);
+  cudaMemcpy(final_host, counter, sizeof(unsigned), cudaMemcpyDeviceToHost);
+  cudaFree(counter);
+  cudaFree(log);
+  cudaFree(ok);
+  cudaMemcpyToSymbol(ra::g_status, &zero, sizeof(int));
+  return st;
 }
 
 // Returns the status word after a wait that runs out: 1 (timeout) expected; also whether

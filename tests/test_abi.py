@@ -25,7 +25,7 @@ def _declared_functions():
 
 def _prob(**kw):
     base = dict(B=1, H=2, n=100, d=64, dtype=ra.RA_BF16, causal=0, rope_base=1e4, pos=None,
-                A1=FAKE, A2=FAKE, A3=FAKE, WQ=FAKE, WK=FAKE, WV=FAKE, E=FAKE)
+                A1=FAKE, A2=FAKE, A3=FAKE, WQ=FAKE, WK=FAKE, WV=FAKE, E=FAKE, deterministic=0)
     base.update(kw)
     return ra.Problem(*(base[f] for f, _ in ra.Problem._fields_))
 
@@ -71,6 +71,7 @@ def test_workspace_bytes():
     (dict(H=-1), ra.RA_ERR_INVALID_ARG),
     (dict(dtype=7), ra.RA_ERR_INVALID_ARG),
     (dict(causal=2), ra.RA_ERR_INVALID_ARG),
+    (dict(deterministic=2), ra.RA_ERR_INVALID_ARG),
     (dict(rope_base=0.0), ra.RA_ERR_INVALID_ARG),
     (dict(rope_base=float("nan")), ra.RA_ERR_INVALID_ARG),
     (dict(A1=None), ra.RA_ERR_INVALID_ARG),

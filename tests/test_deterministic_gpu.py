@@ -1,0 +1,93 @@
+"""The backward's deterministic mode (ra_problem.deterministic = 1).
+
+With it the per-key-tile parts of the query-side gradient are added in a fixed order (key
+tile 0, 1, 2, ... for every query tile), so the weight gradients and the input gradients must
+be bitwise the same on every run, whatever else ran in between; they must still match the
+fp64 oracle at the parity bars.  Without the flag the same sums are formed in arrival order,
+which may differ in the last bits from run to run (not asserted either way).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from test_input_grads_gpu import DA, compare_inputs
+from test_parity_gpu import small, to_device
+from workloads import WORKLOADS, make_inputs
+
+pytestmark = pytest.mark.gpu
+
+OUT = ("dWQ", "dWK", "dWV") + DA
+
+
+def _model(cuda_lib, w, t, deterministic):
+    return cuda_lib.RopeAttention(t["A1"], t["A2"], t["A3"], t["WQ"], t["WK"], t["WV"], t["E"],
+                                  t["pos"], w.causal, w.rope_base, deterministic=deterministic)
+
+
+def _grads(cuda_lib, m, holds):
+    m.forward()
+    if not holds:
+        m.ws.fill_(0xFF)
+    m.backward_inputs(holds)
+    torch.cuda.synchronize()
+    assert cuda_lib.last_error() == cuda_lib.RA_OK
+    out = {k: getattr(m, k).clone() for k in OUT}
+    out["loss"] = float(m.loss.item())
+    return out
+
+
+def _scramble(cuda_lib, dtype):
+    """Another problem's backward in between (other sizes, other causal flag): different
+    timing, L2 contents and counters left in a different workspace."""
+    w = small(dtype, 300, 64, True, B=1, H=2)
+    t = to_device(make_inputs(w, seed=77), dtype)
+    _grads(cuda_lib, _model(cuda_lib, w, t, False), True)
+
+
+def _assert_bitwise(a, b):
+    for k in OUT:
+        x, y = a[k], b[k]
+        assert torch.equal(x.view(torch.int16) if x.dtype == torch.bfloat16 else x.view(torch.int32),
+                           y.view(torch.int16) if y.dtype == torch.bfloat16 else y.view(torch.int32)), k
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("n,d,causal", [(129, 64, True), (385, 128, False), (600, 64, False),
+                                        (1000, 128, True)])
+def test_deterministic_is_bitwise_repeatable_and_matches_the_oracle(cuda_lib, dtype, n, d, causal):
+    w = small(dtype, n, d, causal, B=2, H=2)
+    inp = make_inputs(w, seed=5 + n)
+    t = to_device(inp, dtype)
+    m = _model(cuda_lib, w, t, True)
+    # the same call twice, another problem's backward in between: the same bits.  (Reusing the
+    # forward's workspace and recomputing it are two computations that differ in rounding -
+    # with bf16 I/O delta comes from the fp32 O or from the stored bf16 O - so each is compared
+    # with itself.)
+    runs = {}
+    for holds in (True, True, False, False):
+        runs.setdefault(holds, []).append(_grads(cuda_lib, m, holds))
+        _scramble(cuda_lib, dtype)
+    ref = oracle.forward_backward(inp, w.causal, w.rope_base)
+    for holds, (a, b) in runs.items():
+        _assert_bitwise(a, b)
+        got = {k: a[k].float().cpu().numpy() for k in OUT}
+        got["loss"] = a["loss"]
+        compare_inputs(w, got, ref)
+
+
+def test_deterministic_at_full_size(cuda_lib):
+    """B=2 H=32 n=8192 d=128 causal (bf16): two deterministic steps are bitwise equal and
+    agree with the default mode to within fp32 summation-order effects."""
+    w = WORKLOADS["b2_h32_n8192_d128_bf16_causal"]
+    t = to_device(make_inputs(w), w.dtype)
+    det = _model(cuda_lib, w, t, True)
+    a = _grads(cuda_lib, det, True)
+    _scramble(cuda_lib, w.dtype)
+    b = _grads(cuda_lib, det, True)
+    _assert_bitwise(a, b)
+    c = _grads(cuda_lib, _model(cuda_lib, w, t, False), True)
+    for k in OUT:
+        x, y = a[k].double(), c[k].double()
+        err = float(torch.linalg.vector_norm(x - y) / torch.linalg.vector_norm(y))
+        assert err <= 1e-3, (k, err)

@@ -75,3 +75,30 @@ def test_exp2_poly_against_cuda_exp2f(probe):
                      ctypes.c_void_p(torch.empty_like(low).data_ptr()), 3)
     torch.cuda.synchronize()
     assert torch.isfinite(out).all() and (out >= 0).all() and (out <= 2.0 ** -125).all()
+
+
+def _turns(probe, nblocks, reverse, start, limit_ns):
+    log = (ctypes.c_int * nblocks)()
+    ok = ctypes.c_int(7)
+    final = ctypes.c_uint(0)
+    st = probe.probe_turn(nblocks, reverse, start, ctypes.c_ulonglong(limit_ns), log,
+                          ctypes.byref(ok), ctypes.byref(final))
+    return st, list(log), ok.value, final.value
+
+
+@pytest.mark.parametrize("reverse", [0, 1])
+def test_turn_order(probe, reverse):
+    n = 64
+    st, log, ok, final = _turns(probe, n, reverse, 0, 1_000_000_000)
+    assert st == 0 and ok == 1 and final == n
+    want = list(range(n - 1, -1, -1)) if reverse else list(range(n))
+    assert log == want
+
+
+def test_turn_wait_gives_up(probe):
+    # the counter starts past the only turn there is: the wait must give up, flag a timeout
+    # and still pass the counter on
+    st, log, ok, final = _turns(probe, 1, 0, 3, 20_000_000)
+    assert st == 1 and ok == 0 and final == 4
+    x = torch.ones(4, device="cuda")
+    assert float(x.sum()) == 4.0

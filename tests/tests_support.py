@@ -13,4 +13,8 @@ def probe_lib():
     lib.probe_timeout.restype = ctypes.c_int
     lib.probe_exp2.argtypes = [vp, vp, vp, ctypes.c_int]
     lib.probe_exp2.restype = ctypes.c_int
+    lib.probe_turn.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_uint, ctypes.c_ulonglong,
+                               ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int),
+                               ctypes.POINTER(ctypes.c_uint)]
+    lib.probe_turn.restype = ctypes.c_int
     return lib
