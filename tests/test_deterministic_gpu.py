@@ -53,8 +53,8 @@ def _assert_bitwise(a, b):
 
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
-@pytest.mark.parametrize("n,d,causal", [(129, 64, True), (385, 128, False), (600, 64, False),
-                                        (1000, 128, True)])
+@pytest.mark.parametrize("n,d,causal", [(1, 64, True), (64, 128, False), (129, 64, True),
+                                        (385, 128, False), (600, 64, False), (1000, 128, True)])
 def test_deterministic_is_bitwise_repeatable_and_matches_the_oracle(cuda_lib, dtype, n, d, causal):
     w = small(dtype, n, d, causal, B=2, H=2)
     inp = make_inputs(w, seed=5 + n)
