@@ -139,6 +139,22 @@ ra_status rope_attn_loss_bwd_inputs(const ra_problem* p, const void* O, const fl
                                     int32_t ws_holds_fwd, void* stream);
 
 /*
+ * One step: rope_attn_fwd with the loss, then rope_attn_loss_bwd on the same workspace, in one
+ * call (the page's problem end to end: Loss and its gradient with respect to the weight
+ * matrices, "RoPE Attention kan bijna lineair worden getraind", Probleemdefinitie).
+ *   O, lse       : device, written as by rope_attn_fwd
+ *   loss         : device fp32 scalar (written; may be NULL)
+ *   dWQ/dWK/dWV  : device [H][d][d] fp32 (overwritten)
+ *   ws           : device workspace of at least rope_attn_workspace_bytes(p) bytes
+ * p->E must not be NULL.  The results are those of the two calls (the backward reusing the
+ * forward's intermediates); because the backward follows the forward inside the call, the
+ * backward's recomputation launches are not made at all and the loss is summed once.  The
+ * workspace header ends as after rope_attn_loss_bwd.  Validation and errors as the two calls.
+ */
+ra_status rope_attn_step(const ra_problem* p, void* O, float* lse, float* loss, float* dWQ,
+                         float* dWK, float* dWV, void* ws, size_t ws_bytes, void* stream);
+
+/*
  * One combined weight per head, the parameterisation of the page's problem: the gradient with
  * respect to a single weight x, dLoss/dx = A~^T vec(gamma(x)) ("RoPE Attention kan bijna lineair
  * worden getraind", Probleemdefinitie and Methodologie 1), read as x = vec(X) in the score

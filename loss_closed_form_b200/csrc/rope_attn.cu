@@ -751,6 +751,37 @@ ra_status tc_bwd(const ra_problem* p, const void* O, const float* lse, float* lo
   return launch_status();
 }
 
+// One step on the tensor-core path: the forward with its loss partials, then the backward on
+// the same workspace.  The backward follows the forward inside the call, so its recomputation
+// launches (preparation and projection, gated on the workspace header) are not made at all,
+// and the loss is summed once, by the last launch, which also writes the header.
+ra_status tc_step(const ra_problem* p, void* O, float* lse, float* loss, float* dWQ, float* dWK,
+                  float* dWV, void* ws, cudaStream_t st) {
+  const Layout L = make_layout(p);
+  const ra::WsGate none{nullptr, 0, 0};
+  const int d = p->d;
+  rope_table(p, L, ws, st);
+  ra_status s = d == 128 ? tc_project<128>(p, L, ws, none, false, st)
+                         : tc_project<64>(p, L, ws, none, false, st);
+  if (s != RA_OK) return s;
+  // the forward also zeroes the backward's dQ~ accumulator (p->E is given)
+  s = d == 128 ? tc_fwd_launch<128>(p, L, O, lse, ws, st)
+               : tc_fwd_launch<64>(p, L, O, lse, ws, st);
+  if (s != RA_OK) return s;
+  if (p->deterministic &&
+      cudaMemsetAsync(at<void>(ws, L.turn), 0,
+                      (size_t)p->B * p->H * L.turn_stride * sizeof(unsigned), st) != cudaSuccess)
+    return RA_ERR_CUDA;
+  s = d == 128 ? tc_bwd_launch<128>(p, L, lse, ws, st) : tc_bwd_launch<64>(p, L, lse, ws, st);
+  if (s != RA_OK) return s;
+  ra::WsHeader* stamp = loss ? nullptr : at<ra::WsHeader>(ws, L.hdr);
+  s = d == 128 ? tc_weight_grads<128>(p, L, dWQ, dWK, dWV, ws, stamp, st)
+               : tc_weight_grads<64>(p, L, dWQ, dWK, dWV, ws, stamp, st);
+  if (s != RA_OK) return s;
+  if (loss) finalize(p, L, ws, loss, L.nparts_fwd, none, ra::kWsValid, st);
+  return launch_status();
+}
+
 // ---------------------------------------------------------------------------------------
 // The near-linear approximate method (degree-1 polynomial, low-rank states; fp32 on the CUDA
 // cores).  Workspace: RoPE table, fp32 Q~, K~, V and dQ~, dK~, dV of every instance, the loss
@@ -1097,6 +1128,25 @@ ra_status rope_attn_combined_grad(const float* dWK, int32_t H, int32_t d, float*
   ra::simt::transpose_heads_kernel<<<(unsigned)((total + 255) / 256), 256, 0, st>>>(
       dWK, dX, total, d);
   return launch_status();
+}
+
+ra_status rope_attn_step(const ra_problem* p, void* O, float* lse, float* loss, float* dWQ,
+                         float* dWK, float* dWV, void* ws, size_t ws_bytes, void* stream) {
+  ra_status s = check_problem(p);
+  if (s != RA_OK) return s;
+  if (!p->E || !O || !lse || !dWQ || !dWK || !dWV) return RA_ERR_INVALID_ARG;
+  if (!is_aligned(O, 16) || !is_aligned(lse, 4) || (loss && !is_aligned(loss, 4)) ||
+      !is_aligned(dWQ, 16) || !is_aligned(dWK, 16) || !is_aligned(dWV, 16))
+    return RA_ERR_ALIGNMENT;
+  s = check_ws(p, ws, ws_bytes);
+  if (s != RA_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (p->dtype == RA_F32) {
+    s = simt_fwd<float>(p, O, lse, loss, ws, st);
+    if (s != RA_OK) return s;
+    return simt_bwd(p, O, lse, nullptr, dWQ, dWK, dWV, ws, 1, st);
+  }
+  return tc_step(p, O, lse, loss, dWQ, dWK, dWV, ws, st);
 }
 
 ra_status rope_attn_step_noalloc(const ra_problem* p, void* O, float* lse, float* loss,

@@ -22,7 +22,8 @@ EXPORTED = ("rope_attn_workspace_bytes", "rope_attn_fwd", "rope_attn_loss_bwd",
             "rope_attn_last_error", "rope_attn_status_string", "rope_attn_launch_count",
             "rope_attn_profile_enable", "rope_attn_profile_read", "rope_attn_kernel_name",
             "rope_attn_step_noalloc", "rope_attn_loss_bwd_inputs", "rope_attn_combined_weights",
-            "rope_attn_combined_grad", "rope_attn_approx_workspace_bytes", "rope_attn_approx_step")
+            "rope_attn_combined_grad", "rope_attn_approx_workspace_bytes", "rope_attn_approx_step",
+            "rope_attn_step")
 
 # Capacity of the static scratch behind rope_attn_step_noalloc (RA_NOALLOC_SCRATCH_BYTES).
 NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
@@ -80,6 +81,8 @@ def load() -> ctypes.CDLL:
     lib.rope_attn_kernel_name.restype = ctypes.c_char_p
     lib.rope_attn_step_noalloc.argtypes = [P, vp, vp, vp, vp, vp, vp, vp]
     lib.rope_attn_step_noalloc.restype = ctypes.c_int
+    lib.rope_attn_step.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.rope_attn_step.restype = ctypes.c_int
     lib.rope_attn_loss_bwd_inputs.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz,
                                               i32, vp]
     lib.rope_attn_loss_bwd_inputs.restype = ctypes.c_int
@@ -195,6 +198,16 @@ def combined_grad(dWK, dX, stream=None) -> None:
         raise RopeAttnError(st, "rope_attn_combined_grad")
 
 
+def step(prob: Problem, O, lse, loss, dWQ, dWK, dWV, ws, stream=None) -> None:
+    """rope_attn_step: the forward with the loss and the weight-gradient backward on the same
+    workspace, in one call."""
+    st = load().rope_attn_step(ctypes.byref(prob), _ptr(O), _ptr(lse), _ptr(loss), _ptr(dWQ),
+                               _ptr(dWK), _ptr(dWV), _ptr(ws), ws.numel() * ws.element_size(),
+                               _stream(stream))
+    if st != RA_OK:
+        raise RopeAttnError(st, "rope_attn_step")
+
+
 def step_noalloc(prob: Problem, O, lse, loss, dWQ, dWK, dWV, stream=None) -> None:
     """rope_attn_step_noalloc: forward + backward on the library's static scratch.
 
@@ -307,8 +320,11 @@ class RopeAttention:
         return self.loss, self.dWQ, self.dWK, self.dWV, self.dA1, self.dA2, self.dA3
 
     def step(self, stream=None):
-        self.forward(stream)
-        return self.backward(True, stream)
+        """Forward with the loss, then the weight gradients (rope_attn_step); returns
+        (loss, dWQ, dWK, dWV)."""
+        step(self.prob, self.O, self.lse, self.loss, self.dWQ, self.dWK, self.dWV, self.ws,
+             stream)
+        return self.loss, self.dWQ, self.dWK, self.dWV
 
 
 class RopeAttentionX:

@@ -115,6 +115,26 @@ def test_bwd_argument_errors():
     assert _bwd(p, nbytes=nb - 256) == ra.RA_ERR_WORKSPACE
 
 
+def test_step_argument_errors():
+    """rope_attn_step validates like the forward and the backward together, before anything
+    is launched."""
+    lib = ra.load()
+    p = _prob()
+    nb = lib.rope_attn_workspace_bytes(ctypes.byref(p))
+
+    def call(prob=p, O=FAKE, lse=FAKE, dW=(FAKE, FAKE, FAKE), ws=FAKE * 16, nbytes=nb):
+        return lib.rope_attn_step(ctypes.byref(prob), O, lse, FAKE, *dW, ws, nbytes, None)
+    assert call(prob=_prob(E=None)) == ra.RA_ERR_INVALID_ARG
+    assert call(O=None) == ra.RA_ERR_INVALID_ARG
+    assert call(lse=None) == ra.RA_ERR_INVALID_ARG
+    assert call(dW=(FAKE, FAKE, None)) == ra.RA_ERR_INVALID_ARG
+    assert call(prob=_prob(deterministic=3)) == ra.RA_ERR_INVALID_ARG
+    assert call(dW=(FAKE + 4, FAKE, FAKE)) == ra.RA_ERR_ALIGNMENT
+    assert call(ws=None) == ra.RA_ERR_WORKSPACE
+    assert call(nbytes=nb - 256) == ra.RA_ERR_WORKSPACE
+    assert call(prob=_prob(d=96)) == ra.RA_ERR_UNSUPPORTED
+
+
 def test_bwd_inputs_argument_errors():
     """rope_attn_loss_bwd_inputs validates its extra outputs, then everything the plain
     backward validates, before anything is launched."""
