@@ -28,11 +28,11 @@
 // and beta^T are issued as soon as a buffer's products have completed and its dQ~^T has been
 // read out.
 //
-// Warp roles (448 threads): warps 0-7 softmax / gamma (two warpgroups over the same 128 key
+// Warp roles (480 threads): warps 0-7 softmax / gamma (two warpgroups over the same 128 key
 // rows, each taking half of the 64 query columns) and the epilogue (warps 0-3 dK, 4-7 dV),
 // warps 8-11 drain dQ~ from TMEM into the staging tile (thread 256 issues the bulk
 // reduction), warp 12 TMA producer (it also stages the query tile's lse and delta), warp 13
-// MMA issuer and TMEM owner.
+// issues the gradient products and owns TMEM, warp 14 issues S^T and beta^T.
 #pragma once
 #include "tc_ptx.cuh"
 
@@ -61,8 +61,8 @@ struct BwdCfg {
   static constexpr int LD_OFF = DQS_OFF + DQS;
   static constexpr int BAR_OFF = LD_OFF + NSQ * BQ * 8;
   // kv_full, q_full[NSQ], q_empty[NSQ], s_full[2], pg_full[2], pg_done[2], dq_full[2],
-  // dq_free[2], acc_done, drain, dqs_full, dqs_free, tab_full, ep_full
-  static constexpr int NBAR = 1 + 2 * NSQ + 10 + 6;
+  // dq_free[2], acc_done, drain, dqs_full, dqs_free, tab_full, ep_full, drain2
+  static constexpr int NBAR = 1 + 2 * NSQ + 10 + 7;
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
   static constexpr int SMEM_USED = MISC_OFF + 64;
   static constexpr int SMEM_ALLOC =
@@ -72,8 +72,8 @@ struct BwdCfg {
   static constexpr int TBLK = BK * 128;
   static constexpr int TABT = BK * D * 4;
   static_assert(TABT <= 2 * KTILE && 2 * KTILE <= 2 * NSQ * QTILE, "epilogue staging");
-  static constexpr int THREADS = 448;
-  static constexpr int W_DRAIN = 8, W_PROD = 12, W_MMA = 13;
+  static constexpr int THREADS = 480;
+  static constexpr int W_DRAIN = 8, W_PROD = 12, W_MMA = 13, W_MMA2 = 14;
   // deterministic mode: steps between a query tile's reduction and passing its turn on
   static constexpr int TURN_LAG = 1;
   // TMEM columns: step buffer b at 128 b holds S^T (columns 0-63) and beta^T (64-127); the
@@ -129,6 +129,7 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
   const uint32_t b_dqsfree = smem_u32(&bars[14 + 2 * C::NSQ]);
   const uint32_t b_tab = smem_u32(&bars[15 + 2 * C::NSQ]);  // RoPE rows of the key tile landed
   const uint32_t b_ep = smem_u32(&bars[16 + 2 * C::NSQ]);   // dK / dV staging written
+  const uint32_t b_drain2 = smem_u32(&bars[17 + 2 * C::NSQ]);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   // grid (heads of a group, key tile, group): the CTAs are dispatched x fastest, so each
@@ -161,6 +162,7 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     }
     mbar_init(b_acc, 1);
     mbar_init(b_drain, 1);
+    mbar_init(b_drain2, 1);
     mbar_init(b_dqsfull, 128);
     mbar_init(b_dqsfree, 1);
     mbar_init(b_tab, 1);
@@ -225,12 +227,18 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       for (int ii = (last - C::NSQ + 1 > 0 ? last - C::NSQ + 1 : 0); ii <= last; ++ii)
         mbar_drain(b_qfull(ii % C::NSQ), (ii / C::NSQ) & 1, lim);
     }
-  } else if (warp == C::W_MMA) {
-    // ------------------------------------------------------------------ MMA issuer
-    // per step i in buffer b = i % 2: dV and dK (they read P^T, gamma^T over the S^T columns),
-    // then dQ~^T_i (over the beta^T columns).  S^T of step i + 2 follows as soon as dV and dK
-    // have completed, while dQ~^T_i still runs; beta^T of step i + 2 once the drain has read
-    // dQ~^T_i, while S^T runs: the tensor pipe always has a product queued behind the wait.
+  } else if (warp == C::W_MMA || warp == C::W_MMA2) {
+    // ------------------------------------------------------------------ MMA issuers
+    // Two issuing threads: warp W_MMA2 issues S^T and beta^T of every step, warp W_MMA the
+    // gradient products.  A thread that issues tcgen05.mma is held at each issue until the
+    // tensor pipe takes the product, so with one thread a wait for one chain (the drain
+    // freeing beta^T's columns) also held the other (the next step's products).
+    //   step i, buffer b = i % 2:  S^T_i once dV and dK of step i - 2 have read P^T, gamma^T
+    //   over its columns; beta^T_i once the drain has read dQ~^T_i-2 over its columns;
+    //   dV, dK (P^T, gamma^T from TMEM) then dQ~^T_i (over the beta^T columns, which the
+    //   softmax warps have read) once P^T_i, gamma^T_i are written.
+    // Both poll their barriers: a suspended wait resumes a few hundred cycles after the phase
+    // completes, on the chain every step waits for.
     if (lane == 0) {
       constexpr uint32_t idesc_sb = idesc_bf16_f32(128, C::BQ, false, false);
       constexpr uint32_t idesc_kv = idesc_bf16_f32(128, D, false, true);
@@ -238,79 +246,74 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       // descriptor low words per buffer (sw128_lo), offsets added per K step (sw128_at)
       const uint32_t ka_k = sw128_lo(sbase + C::K_OFF, 16), va_k = sw128_lo(sbase + C::V_OFF, 16);
       const uint32_t ka_mn = sw128_lo(sbase + C::K_OFF, C::KBLK);
-      bool ok = mbar_wait(b_kv, 0, abort_flag, lim);
-      // S^T (z = 0) or beta^T (z = 1) of step ii into its buffer
-      auto issue_sb = [&](int ii, int z) {
-        const int s = ii % C::NSQ;
-        const uint32_t ab = z ? va_k : ka_k;
-        const uint32_t bb = sw128_lo(sbase + (z ? C::L_OFF : C::Q_OFF) + s * C::QTILE, 16);
-        const uint32_t d_acc = tmem + (ii & 1) * C::T_BUF + (z ? C::T_B : 0);
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t ko = (kk >> 2) * C::KBLK + (kk & 3) * 32;
-          const uint32_t qo = (kk >> 2) * C::QBLK + (kk & 3) * 32;
-          mma_ss(d_acc, sw128_at(ab, ko), sw128_at(bb, qo), idesc_sb, kk > 0);
-        }
-      };
-      auto wait_q = [&](int ii) -> bool {
-        if (!mbar_wait(b_qfull(ii % C::NSQ), (ii / C::NSQ) & 1, abort_flag, lim)) return false;
-        tc_fence_after();
-        return true;
-      };
+      bool ok = mbar_wait_poll(b_kv, 0, abort_flag, lim);
       tc_fence_after();
-      for (int ii = 0; ok && ii < 2 && ii < NI; ++ii) {
-        if (!(ok = wait_q(ii))) break;
-        issue_sb(ii, 0);
-        issue_sb(ii, 1);
-        mma_commit(b_sfull(ii));
-      }
-      for (int ii = 0; ok && ii < NI; ++ii) {
-        const int s = ii % C::NSQ, b = ii & 1;
-        const uint32_t ph = (ii >> 1) & 1;
-        if (!(ok = mbar_wait(b_pgfull(b), ph, abort_flag, lim))) break;
-        tc_fence_after();
-        const uint32_t buf = tmem + b * C::T_BUF;
-        // dV += P^T l_i, dK += gamma^T Q~_i: M = 128 keys, N = D, K = 64 queries, with P^T and
-        // gamma^T read from TMEM (two bf16 per column, 8 columns per K step of 16 queries:
-        // queries 16 kk .. of warpgroup kk / 2 at 32 (kk / 2) + 8 (kk % 2))
-        const uint32_t qb_mn = sw128_lo(sbase + C::Q_OFF + s * C::QTILE, C::QBLK);
-        const uint32_t lb_mn = sw128_lo(sbase + C::L_OFF + s * C::QTILE, C::QBLK);
+      if (warp == C::W_MMA2) {
+        // S^T (z = 0) or beta^T (z = 1) of step ii into its buffer
+        auto issue_sb = [&](int ii, int z) {
+          const int s = ii % C::NSQ;
+          const uint32_t ab = z ? va_k : ka_k;
+          const uint32_t bb = sw128_lo(sbase + (z ? C::L_OFF : C::Q_OFF) + s * C::QTILE, 16);
+          const uint32_t d_acc = tmem + (ii & 1) * C::T_BUF + (z ? C::T_B : 0);
 #pragma unroll
-        for (int kk = 0; kk < C::BQ / 16; ++kk) {
-          const uint32_t pa = buf + 32 * (kk >> 1) + 8 * (kk & 1);
-          mma_ts(tmem + C::T_DV, pa, sw128_at(lb_mn, kk * 2048), idesc_kv, (ii > 0 || kk > 0));
-          mma_ts(tmem + C::T_DK, pa + C::T_GT, sw128_at(qb_mn, kk * 2048), idesc_kv,
-                 (ii > 0 || kk > 0));
-        }
-        mma_commit(b_pgdone(b));
-        mma_commit(b_qempty(s));
-        // dQ~_i^T = K~^T gamma^T (M = D, N = 64 queries, K = 128 keys) over the columns beta^T
-        // held (the softmax warps have read them)
-        const uint32_t gt_mn = sw128_lo(sbase + C::G_OFF + b * C::PG, C::KBLK);
-#pragma unroll
-        for (int kk = 0; kk < C::BK / 16; ++kk)
-          mma_ss(buf + C::T_DQ, sw128_at(ka_mn, kk * 2048), sw128_at(gt_mn, kk * 2048), idesc_dq,
-                 kk > 0);
-        mma_commit(b_dqfull(b));
-        if (ii + 2 < NI) {
-          // S^T_i+2 over P^T, gamma^T once dV and dK have read them; beta^T_i+2 over dQ~^T_i
-          // once the drain has read it (gamma^T slot b, read by dQ~^T_i, is rewritten only
-          // after sfull, which follows beta^T)
-          if (!(ok = wait_q(ii + 2))) break;
-          if (!(ok = mbar_wait(b_pgdone(b), ph, abort_flag, lim))) break;
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t ko = (kk >> 2) * C::KBLK + (kk & 3) * 32;
+            const uint32_t qo = (kk >> 2) * C::QBLK + (kk & 3) * 32;
+            mma_ss(d_acc, sw128_at(ab, ko), sw128_at(bb, qo), idesc_sb, kk > 0);
+          }
+        };
+        for (int ii = 0; ok && ii < NI; ++ii) {
+          const int b = ii & 1;
+          const uint32_t pph = ((ii - 2) >> 1) & 1;  // phase of step ii - 2 in buffer b
+          const int s = ii % C::NSQ;
+          if (!(ok = mbar_wait_poll(b_qfull(s), (ii / C::NSQ) & 1, abort_flag, lim))) break;
+          if (ii >= 2 && !(ok = mbar_wait_poll(b_pgdone(b), pph, abort_flag, lim))) break;
           tc_fence_after();
-          issue_sb(ii + 2, 0);
-          if (!(ok = mbar_wait(b_dqfree(b), ph, abort_flag, lim))) break;
+          issue_sb(ii, 0);
+          if (ii >= 2 && !(ok = mbar_wait_poll(b_dqfree(b), pph, abort_flag, lim))) break;
           tc_fence_after();
-          issue_sb(ii + 2, 1);
+          issue_sb(ii, 1);
           mma_commit(b_sfull(b));
         }
-      }
-      if (ok) {
-        mma_commit(b_acc);
+        if (!ok) {
+          mma_commit(b_drain2);
+          mbar_drain(b_drain2, 0, lim);
+        }
       } else {
-        mma_commit(b_drain);
-        mbar_drain(b_drain, 0, lim);
+        for (int ii = 0; ok && ii < NI; ++ii) {
+          const int s = ii % C::NSQ, b = ii & 1;
+          if (!(ok = mbar_wait_poll(b_pgfull(b), (ii >> 1) & 1, abort_flag, lim))) break;
+          tc_fence_after();
+          const uint32_t buf = tmem + b * C::T_BUF;
+          // dV += P^T l_i, dK += gamma^T Q~_i: M = 128 keys, N = D, K = 64 queries, with P^T
+          // and gamma^T read from TMEM (two bf16 per column, 8 columns per K step of 16
+          // queries: queries 16 kk .. of warpgroup kk / 2 at 32 (kk / 2) + 8 (kk % 2))
+          const uint32_t qb_mn = sw128_lo(sbase + C::Q_OFF + s * C::QTILE, C::QBLK);
+          const uint32_t lb_mn = sw128_lo(sbase + C::L_OFF + s * C::QTILE, C::QBLK);
+#pragma unroll
+          for (int kk = 0; kk < C::BQ / 16; ++kk) {
+            const uint32_t pa = buf + 32 * (kk >> 1) + 8 * (kk & 1);
+            mma_ts(tmem + C::T_DV, pa, sw128_at(lb_mn, kk * 2048), idesc_kv, (ii > 0 || kk > 0));
+            mma_ts(tmem + C::T_DK, pa + C::T_GT, sw128_at(qb_mn, kk * 2048), idesc_kv,
+                   (ii > 0 || kk > 0));
+          }
+          mma_commit(b_pgdone(b));
+          mma_commit(b_qempty(s));
+          // dQ~_i^T = K~^T gamma^T (M = D, N = 64 queries, K = 128 keys) over the columns
+          // beta^T held
+          const uint32_t gt_mn = sw128_lo(sbase + C::G_OFF + b * C::PG, C::KBLK);
+#pragma unroll
+          for (int kk = 0; kk < C::BK / 16; ++kk)
+            mma_ss(buf + C::T_DQ, sw128_at(ka_mn, kk * 2048), sw128_at(gt_mn, kk * 2048),
+                   idesc_dq, kk > 0);
+          mma_commit(b_dqfull(b));
+        }
+        if (ok) {
+          mma_commit(b_acc);
+        } else {
+          mma_commit(b_drain);
+          mbar_drain(b_drain, 0, lim);
+        }
       }
     }
   } else if (warp < C::W_DRAIN) {
@@ -455,7 +458,8 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     int passed = 0;  // query tiles whose turn this key tile has passed on (deterministic mode)
     for (int ii = 0; ii < NI; ++ii) {
       const int b = ii & 1;
-      if (!mbar_wait_warp(b_dqfull(b), (ii >> 1) & 1, abort_flag, lim)) break;
+      // polled: the MMA issuer waits for this drain before it can issue beta^T two steps on
+      if (!mbar_wait_warp_poll(b_dqfull(b), (ii >> 1) & 1, abort_flag, lim)) break;
       tc_fence_after();
       uint32_t r0[32], r1[32];
       const uint32_t dq = tmem + lane_base + b * C::T_BUF + C::T_DQ;

@@ -101,6 +101,44 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint32_
   }
 }
 
+// Non-blocking test of the same phase.
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// mbar_wait by polling with test_wait (no suspension, so the thread sees the phase complete
+// within a few cycles; it keeps taking issue slots while it waits).  Same limits and abort
+// behaviour; the flag and the clock are checked every 256 polls.
+__device__ __forceinline__ bool mbar_wait_poll(uint32_t bar, uint32_t parity, uint32_t abort_flag,
+                                               uint64_t limit_ns) {
+  if (mbar_test_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_test_wait(bar, parity)) return true;
+    if ((it & 255u) == 0) {
+      if (abort_get(abort_flag)) return false;
+      if (globaltimer() - t0 > limit_ns) {
+        flag_error(kDevTimeout);
+        abort_set(abort_flag, 1);
+        return false;
+      }
+    }
+  }
+}
+__device__ __forceinline__ bool mbar_wait_warp_poll(uint32_t bar, uint32_t parity,
+                                                    uint32_t abort_flag, uint64_t limit_ns) {
+  const bool ok = mbar_wait_poll(bar, parity, abort_flag, limit_ns);
+  return __all_sync(0xffffffffu, ok);
+}
+
 // Warp-uniform form: every lane of the calling warp must call it; true only if the wait
 // succeeded for all lanes (so .sync.aligned TMEM instructions that follow stay convergent).
 __device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity, uint32_t abort_flag,
