@@ -218,6 +218,14 @@ int64_t rope_attn_launch_count(void);
 void rope_attn_profile_enable(int32_t on);
 
 /*
+ * Restricts those events to the launches of kernel id `kernel_id` (see rope_attn_kernel_name);
+ * a negative or out-of-range id restores events around every launch (the default).  Each
+ * event pair adds a few microseconds between two dependent launches, so a timed region that
+ * needs one kernel's duration brackets that kernel alone.
+ */
+void rope_attn_profile_only(int32_t kernel_id);
+
+/*
  * Waits for the recorded events, then writes for each kernel id k < max_kernels the summed
  * device time in milliseconds (ms[k]) and the number of launches (launches[k]) since the
  * last read, and clears the records.  Returns the number of kernel ids (see

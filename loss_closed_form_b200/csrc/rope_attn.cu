@@ -68,6 +68,7 @@ struct ProfRecord {
 };
 struct Profiler {
   bool on = false;
+  int only = -1;  // >= 0: only this kernel's launches get events
   std::vector<ProfRecord> recs;
   std::vector<cudaEvent_t> pool;
   cudaEvent_t get() {
@@ -96,7 +97,7 @@ struct Launch {
   int slot = -1;
   Launch(KernelId id, cudaStream_t s) : st(s) {
     ++t_launches;
-    if (t_prof.on) {
+    if (t_prof.on && (t_prof.only < 0 || t_prof.only == id)) {
       ProfRecord r{id, t_prof.get(), t_prof.get()};
       cudaEventRecord(r.start, st);
       t_prof.recs.push_back(r);
@@ -1234,6 +1235,10 @@ int64_t rope_attn_launch_count(void) {
 void rope_attn_profile_enable(int32_t on) {
   t_prof.on = on != 0;
   if (!t_prof.on) t_prof.recycle();
+}
+
+void rope_attn_profile_only(int32_t kernel_id) {
+  t_prof.only = (kernel_id >= 0 && kernel_id < K_COUNT) ? kernel_id : -1;
 }
 
 int32_t rope_attn_profile_read(float* ms, int32_t* launches, int32_t max_kernels) {

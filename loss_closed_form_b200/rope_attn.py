@@ -20,7 +20,8 @@ RA_F32, RA_BF16 = 0, 1
 # Every symbol include/rope_attn.h declares.
 EXPORTED = ("rope_attn_workspace_bytes", "rope_attn_fwd", "rope_attn_loss_bwd",
             "rope_attn_last_error", "rope_attn_status_string", "rope_attn_launch_count",
-            "rope_attn_profile_enable", "rope_attn_profile_read", "rope_attn_kernel_name",
+            "rope_attn_profile_enable", "rope_attn_profile_only", "rope_attn_profile_read",
+            "rope_attn_kernel_name",
             "rope_attn_step_noalloc", "rope_attn_loss_bwd_inputs", "rope_attn_combined_weights",
             "rope_attn_combined_grad", "rope_attn_approx_workspace_bytes", "rope_attn_approx_step",
             "rope_attn_step")
@@ -75,6 +76,8 @@ def load() -> ctypes.CDLL:
     lib.rope_attn_launch_count.restype = ctypes.c_int64
     lib.rope_attn_profile_enable.argtypes = [i32]
     lib.rope_attn_profile_enable.restype = None
+    lib.rope_attn_profile_only.argtypes = [i32]
+    lib.rope_attn_profile_only.restype = None
     lib.rope_attn_profile_read.argtypes = [vp, vp, i32]
     lib.rope_attn_profile_read.restype = i32
     lib.rope_attn_kernel_name.argtypes = [i32]
@@ -244,6 +247,12 @@ def launch_count() -> int:
 
 def profile_enable(on: bool) -> None:
     load().rope_attn_profile_enable(int(bool(on)))
+
+
+def profile_only(kernel: str = None) -> None:
+    """Events around the launches of the named kernel only (None: around every launch)."""
+    kid = -1 if kernel is None else kernel_names().index(kernel)
+    load().rope_attn_profile_only(kid)
 
 
 def profile_read(max_kernels: int = 64):
