@@ -335,6 +335,22 @@ bool map_f32_rows_sw128(CUtensorMap* m, void* base, uint64_t cols, uint64_t rows
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 3-D map over fp32 rows [outer][rows][cols] with boxes of 32 columns (128 bytes) x box_rows,
+// 128-byte swizzle (the target of the d = 64 backward's bulk reductions, staged as swizzled
+// rows so that one thread per row writes without bank conflicts).
+bool map_f32_3d_sw128(CUtensorMap* m, void* base, uint64_t cols, uint64_t rows, uint64_t outer,
+                      uint32_t box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {cols, rows, outer};
+  cuuint64_t strides[2] = {cols * 4, rows * cols * 4};
+  cuuint32_t box[3] = {32, box_rows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base, dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // 3-D map over fp32 rows [outer][rows][cols] with a box of cols x box_rows, no swizzle
 // (the target of bulk reductions).
 bool map_f32_3d(CUtensorMap* m, void* base, uint64_t cols, uint64_t rows, uint64_t outer,
@@ -657,7 +673,8 @@ ra_status tc_bwd_launch(const ra_problem* p, const Layout& L, const float* lse, 
       !map_bf16_3d(&mk, at<void>(ws, L.kt), D, n, BH, C::BK) ||
       !map_bf16_3d(&mv, at<void>(ws, L.v), D, n, BH, C::BK) ||
       !map_bf16_3d(&ml, at<void>(ws, L.ell), D, n, BH, C::BQ) ||
-      !map_f32_3d(&mdq, at<void>(ws, L.dqt), D, n, BH, C::BQ) ||
+      !(C::PAIR ? map_f32_3d_sw128(&mdq, at<void>(ws, L.dqt), D, n, BH, C::BQ)
+                : map_f32_3d(&mdq, at<void>(ws, L.dqt), D, n, BH, C::BQ)) ||
       !map_f32_rows_sw128(&mtab, at<void>(ws, L.rope), D, n, C::BK) ||
       !map_bf16_3d(&mdk, at<void>(ws, L.dk16), D, n, BH, C::BK) ||
       !map_bf16_3d(&mdv, at<void>(ws, L.dv16), D, n, BH, C::BK))

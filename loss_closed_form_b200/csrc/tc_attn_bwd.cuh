@@ -50,13 +50,22 @@ struct BwdCfg {
   static constexpr int KBLK = BK * 128;       // one swizzle block of a 128-row tile
   static constexpr int QBLK = BQ * 128;       // one swizzle block of a 64-row tile
   static constexpr int PG = BK * BQ * 2;      // gamma^T buffer bytes (one swizzle block)
+  // d = 64: dQ~ of two consecutive query tiles in one product, dQ~ = gamma K~ with the 128
+  // queries on TMEM lanes (M = 128; the transposed product would have M = d = 64, which
+  // takes a tensor-core instruction as long as M = 128 does), accumulated in TMEM columns of
+  // its own.  d = 128 has no free columns and keeps one dQ~^T = K~^T gamma^T per tile.
+  static constexpr bool PAIR = (D == 64);
+  static constexpr int NG = PAIR ? 4 : 2;     // gamma^T slots
   static constexpr int K_OFF = 0;
   static constexpr int V_OFF = K_OFF + KTILE;
   static constexpr int Q_OFF = V_OFF + KTILE;            // NSQ stages
   static constexpr int L_OFF = Q_OFF + NSQ * QTILE;      // NSQ stages
-  static constexpr int G_OFF = L_OFF + NSQ * QTILE;      // gamma^T [2], B operand of dQ~^T
-  static constexpr int DQS_OFF = G_OFF + 2 * PG;          // fp32 [BQ][D] dQ~ staging tile
-  static constexpr int DQS = BQ * D * 4;
+  static constexpr int G_OFF = L_OFF + NSQ * QTILE;      // gamma^T [NG], an operand of dQ~
+  // fp32 dQ~ staging: [BQ][D] row-major (d = 128), or per pair two halves (one per query
+  // tile) of two [64 rows][32 columns] boxes in the 128-byte swizzle (d = 64)
+  static constexpr int DQS_OFF = G_OFF + NG * PG;
+  static constexpr int DQS = (PAIR ? 2 : 1) * BQ * D * 4;
+  static constexpr int DQ_HALF = BQ * D * 4, DQ_BOX = BQ * 32 * 4;
   // float [NSQ][BQ / 2][4]: (-lse * log2(e) of rows 2i, 2i + 1, delta of rows 2i, 2i + 1)
   static constexpr int LD_OFF = DQS_OFF + DQS;
   static constexpr int BAR_OFF = LD_OFF + NSQ * BQ * 8;
@@ -81,7 +90,10 @@ struct BwdCfg {
   // bf16 per column) and dQ~^T is accumulated at 64
   static constexpr uint32_t T_BUF = 128, T_B = 64, T_DQ = 64, T_GT = 16, T_DK = 256,
                             T_DV = 256 + D;
+  // d = 64: the pair products' dQ~ (128 query lanes x 64 columns) in two buffers
+  static constexpr uint32_t T_DQP = 256 + 2 * D;
   static constexpr uint32_t T_COLS = 512;
+  static_assert(!PAIR || T_DQP + 2 * D <= T_COLS, "TMEM budget");
   static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
 };
 
@@ -270,7 +282,8 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
           if (ii >= 2 && !(ok = mbar_wait_poll(b_pgdone(b), pph, abort_flag, lim))) break;
           tc_fence_after();
           issue_sb(ii, 0);
-          if (ii >= 2 && !(ok = mbar_wait_poll(b_dqfree(b), pph, abort_flag, lim))) break;
+          if (!C::PAIR && ii >= 2 && !(ok = mbar_wait_poll(b_dqfree(b), pph, abort_flag, lim)))
+            break;
           tc_fence_after();
           issue_sb(ii, 1);
           mma_commit(b_sfull(b));
@@ -299,14 +312,34 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
           }
           mma_commit(b_pgdone(b));
           mma_commit(b_qempty(s));
-          // dQ~_i^T = K~^T gamma^T (M = D, N = 64 queries, K = 128 keys) over the columns
-          // beta^T held
-          const uint32_t gt_mn = sw128_lo(sbase + C::G_OFF + b * C::PG, C::KBLK);
+          if constexpr (!C::PAIR) {
+            // dQ~_i^T = K~^T gamma^T (M = D, N = 64 queries, K = 128 keys) over the columns
+            // beta^T held
+            const uint32_t gt_mn = sw128_lo(sbase + C::G_OFF + b * C::PG, C::KBLK);
 #pragma unroll
-          for (int kk = 0; kk < C::BK / 16; ++kk)
-            mma_ss(buf + C::T_DQ, sw128_at(ka_mn, kk * 2048), sw128_at(gt_mn, kk * 2048),
-                   idesc_dq, kk > 0);
-          mma_commit(b_dqfull(b));
+            for (int kk = 0; kk < C::BK / 16; ++kk)
+              mma_ss(buf + C::T_DQ, sw128_at(ka_mn, kk * 2048), sw128_at(gt_mn, kk * 2048),
+                     idesc_dq, kk > 0);
+            mma_commit(b_dqfull(b));
+          } else if ((ii & 1) || ii == NI - 1) {
+            // dQ~ of query tiles 2 pr and 2 pr + 1 = gamma K~: M = 128 queries (A: the two
+            // gamma^T slots, query-contiguous, 64 queries apart by PG), N = D, K = 128 keys
+            // (B: K~, d-contiguous).  When NI is odd, the last product's rows 64-127 read a
+            // stale slot and are not reduced.  Its buffer is free once the drain has read
+            // pair pr - 2.
+            constexpr uint32_t idesc_dqp = idesc_bf16_f32(128, D, true, true);
+            const int pr = ii >> 1, pb = pr & 1;
+            if (pr >= 2 && !(ok = mbar_wait_poll(b_dqfree(pb), ((pr - 2) >> 1) & 1, abort_flag,
+                                                 lim)))
+              break;
+            tc_fence_after();
+            const uint32_t ga = sw128_lo(sbase + C::G_OFF + ((2 * pr) % C::NG) * C::PG, C::PG);
+#pragma unroll
+            for (int kk = 0; kk < C::BK / 16; ++kk)
+              mma_ss(tmem + C::T_DQP + pb * D, sw128_at(ga, kk * 2048),
+                     sw128_at(ka_mn, kk * 2048), idesc_dqp, kk > 0);
+            mma_commit(b_dqfull(pb));
+          }
         }
         if (ok) {
           mma_commit(b_acc);
@@ -371,11 +404,12 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         }
       }
       // P^T and gamma^T over the S^T columns this warpgroup has just read (the products of
-      // step i - 2, which read this buffer and gamma^T slot b, completed before S^T of step i
-      // was issued)
+      // step i - 2, which read this buffer and gamma^T slot i % NG, completed before S^T of
+      // step i was issued; at d = 64 the pair product that read the slot was issued before
+      // dV and dK of step i - 2, whose completion S^T of step i waits for)
       tmem_st16(buf, pw);
       tmem_st16(buf + C::T_GT, gw);
-      const uint32_t gsm = sbase + C::G_OFF + b * C::PG;
+      const uint32_t gsm = sbase + C::G_OFF + (ii % C::NG) * C::PG;
 #pragma unroll
       for (int c8 = 0; c8 < 4; ++c8)
         st_shared_v4(gsm + sw128_offset(row, 4 * half + c8), gw[4 * c8], gw[4 * c8 + 1],
@@ -449,75 +483,143 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     // ------------------------------------------------------------------ dQ~ drain (warps 8-11)
     const int wq = warp - C::W_DRAIN;
     const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
-    // accumulator row (head-dimension index) held by this lane: M = 128 puts row r in lane r,
-    // M = 64 puts row r in lane (r % 16) + 32 (r / 16)
-    const int drow = (D == 128) ? (wq * 32 + lane) : (wq * 16 + lane);
-    const bool has_row = (D == 128) || lane < 16;
     const uint32_t stage = sbase + C::DQS_OFF;
     const bool issuer = tid == 32 * C::W_DRAIN;
     int passed = 0;  // query tiles whose turn this key tile has passed on (deterministic mode)
-    for (int ii = 0; ii < NI; ++ii) {
-      const int b = ii & 1;
-      // polled: the MMA issuer waits for this drain before it can issue beta^T two steps on
-      if (!mbar_wait_warp_poll(b_dqfull(b), (ii >> 1) & 1, abort_flag, lim)) break;
-      tc_fence_after();
-      uint32_t r0[32], r1[32];
-      const uint32_t dq = tmem + lane_base + b * C::T_BUF + C::T_DQ;
-      tmem_ld32(dq, r0);
-      tmem_ld32(dq + 32, r1);
-      tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive(b_dqfree(b));
-      // the staging tile is free once the previous bulk reduction has read it
-      if (!mbar_wait_warp(b_dqsfree, (ii & 1) ^ 1, abort_flag, lim)) break;
-      if (has_row) {
-        // row-major [q][d] fp32: for one q the lanes write consecutive d
-#pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          st_shared_f32(stage + (c * D + drow) * 4, __uint_as_float(r0[c]));
-          st_shared_f32(stage + ((32 + c) * D + drow) * 4, __uint_as_float(r1[c]));
+    if constexpr (!C::PAIR) {
+      // accumulator row (head-dimension index) held by this lane: M = 128 puts row r in lane
+      // r, M = 64 puts row r in lane (r % 16) + 32 (r / 16)
+      const int drow = (D == 128) ? (wq * 32 + lane) : (wq * 16 + lane);
+      const bool has_row = (D == 128) || lane < 16;
+      for (int ii = 0; ii < NI; ++ii) {
+        const int b = ii & 1;
+        // polled: the MMA issuer waits for this drain before it can issue beta^T two steps on
+        if (!mbar_wait_warp_poll(b_dqfull(b), (ii >> 1) & 1, abort_flag, lim)) break;
+        tc_fence_after();
+        uint32_t r0[32], r1[32];
+        const uint32_t dq = tmem + lane_base + b * C::T_BUF + C::T_DQ;
+        tmem_ld32(dq, r0);
+        tmem_ld32(dq + 32, r1);
+        tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(b_dqfree(b));
+        // the staging tile is free once the previous bulk reduction has read it
+        if (!mbar_wait_warp(b_dqsfree, (ii & 1) ^ 1, abort_flag, lim)) break;
+        if (has_row) {
+          // row-major [q][d] fp32: for one q the lanes write consecutive d
+  #pragma unroll
+          for (int c = 0; c < 32; ++c) {
+            st_shared_f32(stage + (c * D + drow) * 4, __uint_as_float(r0[c]));
+            st_shared_f32(stage + ((32 + c) * D + drow) * 4, __uint_as_float(r1[c]));
+          }
         }
-      }
-      fence_proxy_async_smem();
-      mbar_arrive(b_dqsfull);
-      bool iok = true;
-      if (issuer) {
-        iok = mbar_wait(b_dqsfull, ii & 1, abort_flag, lim);
-        if (iok && p.turn) {
-          // deterministic mode: query tile q gets the parts of key tiles kmax(q), kmax(q) - 1,
-          // ..., 0 in that order (all of them contribute to it), so key tile kt adds its part
-          // once kmax(q) - kt others have.  Those others were dispatched before this CTA and
-          // reach q two query tiles sooner.  The turn of a tile passes on once its reduction
-          // has landed, checked TURN_LAG steps later (when at most the TURN_LAG newer ones are
-          // in flight: the key tile after this one in the order reaches q later still).
-          const int q = i_start + ii;
-          const int kmax = p.causal ? min(p.nk - 1, (q * C::BQ + C::BQ - 1) / C::BK) : p.nk - 1;
-          unsigned* tc = p.turn + (size_t)bh * p.turn_stride + q;
-          if (turn_wait(tc, static_cast<unsigned>(kmax - kt), lim)) {
-            fence_proxy_async_global();
+        fence_proxy_async_smem();
+        mbar_arrive(b_dqsfull);
+        bool iok = true;
+        if (issuer) {
+          iok = mbar_wait(b_dqsfull, ii & 1, abort_flag, lim);
+          if (iok && p.turn) {
+            // deterministic mode: query tile q gets the parts of key tiles kmax(q), kmax(q) - 1,
+            // ..., 0 in that order (all of them contribute to it), so key tile kt adds its part
+            // once kmax(q) - kt others have.  Those others were dispatched before this CTA and
+            // reach q two query tiles sooner.  The turn of a tile passes on once its reduction
+            // has landed, checked TURN_LAG steps later (when at most the TURN_LAG newer ones are
+            // in flight: the key tile after this one in the order reaches q later still).
+            const int q = i_start + ii;
+            const int kmax = p.causal ? min(p.nk - 1, (q * C::BQ + C::BQ - 1) / C::BK) : p.nk - 1;
+            unsigned* tc = p.turn + (size_t)bh * p.turn_stride + q;
+            if (turn_wait(tc, static_cast<unsigned>(kmax - kt), lim)) {
+              fence_proxy_async_global();
+              tma_reduce_add_3d(&tm_dq, stage, 0, (i_start + ii) * C::BQ, bh);
+              bulk_commit();
+              bulk_wait_read0();
+              mbar_arrive(b_dqsfree);
+              if (passed <= ii - C::TURN_LAG) {
+                bulk_wait_n<C::TURN_LAG>();
+                fence_proxy_async_global();
+                turn_pass(tc - (ii - passed));
+                ++passed;
+              }
+            } else {
+              abort_set(abort_flag, 1);  // given up: the turns still pass, the status says so
+              iok = false;
+              mbar_arrive(b_dqsfree);
+            }
+          } else if (iok) {
             tma_reduce_add_3d(&tm_dq, stage, 0, (i_start + ii) * C::BQ, bh);
             bulk_commit();
             bulk_wait_read0();
             mbar_arrive(b_dqsfree);
-            if (passed <= ii - C::TURN_LAG) {
+          }
+        }
+        if (!__all_sync(0xffffffffu, iok)) break;  // leave the loop together
+      }
+    } else {
+      // d = 64: one pair of query tiles per product, lanes = queries 0-127 of the pair (tiles
+      // 2 pr, 2 pr + 1), 64 columns = d.  Each lane writes its row as 16-byte chunks in the
+      // 128-byte swizzle (chunk j of row q at j ^ (q % 8)), so a warp's stores spread over
+      // all banks; each query tile then leaves as two [64 rows][32 columns] reductions.
+      int issued = 0;  // query tiles whose reduction has been issued
+      const int NP = (NI + 1) / 2;
+      const int q = wq * 32 + lane;
+      const uint32_t qrow = stage + (q >> 6) * C::DQ_HALF + (q & 63) * 128;
+      const uint32_t sw = static_cast<uint32_t>(q & 7);
+      for (int pr = 0; pr < NP; ++pr) {
+        const int pb = pr & 1;
+        if (!mbar_wait_warp_poll(b_dqfull(pb), (pr >> 1) & 1, abort_flag, lim)) break;
+        tc_fence_after();
+        uint32_t r0[32], r1[32];
+        const uint32_t dq = tmem + lane_base + C::T_DQP + pb * D;
+        tmem_ld32(dq, r0);
+        tmem_ld32(dq + 32, r1);
+        tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(b_dqfree(pb));
+        // the staging tile is free once the previous bulk reductions have read it
+        if (!mbar_wait_warp(b_dqsfree, (pr & 1) ^ 1, abort_flag, lim)) break;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const uint32_t off = (static_cast<uint32_t>(j) ^ sw) << 4;
+          st_shared_v4(qrow + off, r0[4 * j], r0[4 * j + 1], r0[4 * j + 2], r0[4 * j + 3]);
+          st_shared_v4(qrow + C::DQ_BOX + off, r1[4 * j], r1[4 * j + 1], r1[4 * j + 2],
+                       r1[4 * j + 3]);
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(b_dqsfull);
+        bool iok = true;
+        if (issuer) {
+          iok = mbar_wait(b_dqsfull, pr & 1, abort_flag, lim);
+          for (int h = 0; iok && h < 2 && 2 * pr + h < NI; ++h) {
+            const int qt = i_start + 2 * pr + h;
+            if (p.turn) {
+              // deterministic mode: as for d = 128 above, per query tile
+              const int kmax = p.causal ? min(p.nk - 1, (qt * C::BQ + C::BQ - 1) / C::BK)
+                                        : p.nk - 1;
+              unsigned* tc = p.turn + (size_t)bh * p.turn_stride + qt;
+              if (!turn_wait(tc, static_cast<unsigned>(kmax - kt), lim)) {
+                abort_set(abort_flag, 1);  // given up: the turns still pass, the status says so
+                iok = false;
+                break;
+              }
+              fence_proxy_async_global();
+            }
+            const uint32_t src = stage + h * C::DQ_HALF;
+            tma_reduce_add_3d(&tm_dq, src, 0, qt * C::BQ, bh);
+            tma_reduce_add_3d(&tm_dq, src + C::DQ_BOX, 32, qt * C::BQ, bh);
+            bulk_commit();
+            ++issued;
+            while (p.turn && passed + C::TURN_LAG < issued) {
               bulk_wait_n<C::TURN_LAG>();
               fence_proxy_async_global();
-              turn_pass(tc - (ii - passed));
+              turn_pass(p.turn + (size_t)bh * p.turn_stride + i_start + passed);
               ++passed;
             }
-          } else {
-            abort_set(abort_flag, 1);  // given up: the turns still pass, the status says so
-            iok = false;
-            mbar_arrive(b_dqsfree);
           }
-        } else if (iok) {
-          tma_reduce_add_3d(&tm_dq, stage, 0, (i_start + ii) * C::BQ, bh);
-          bulk_commit();
           bulk_wait_read0();
           mbar_arrive(b_dqsfree);
         }
+        if (!__all_sync(0xffffffffu, iok)) break;  // leave the loop together
       }
-      if (!__all_sync(0xffffffffu, iok)) break;  // leave the loop together
     }
     if (issuer) bulk_wait_read0();  // the reductions have read the staging tile
     if (issuer && p.turn) {
