@@ -7,6 +7,9 @@
 //   must give up, record a timeout in the status word and return (no trap, no hang).
 // probe_turn: the turn counters of the ordered (deterministic) accumulation: CTAs take turns
 //   in a given order and log it, or one waits for a turn that never comes and gives up.
+// probe_mma_rate: how long one tcgen05.mma (K = 16) of a given shape holds the tensor pipe
+//   when one or two threads of a CTA issue them back to back, one CTA per SM (clock64 around
+//   the issue loop and the completion; the operands are zeros).
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -179,6 +182,69 @@ __global__ void probe_exp2_kernel(const float* __restrict__ x, float* __restrict
   ref[i] = exp2f(x[i]);
 }
 
+
+// One CTA per SM; warps w < nissuers each issue nmma products of shape M x N x 16 (A from
+// shared memory, or from TMEM when a_tmem) into their own accumulator, then wait for them.
+// cycles[cta] = clock64 from the first issue to the last completion seen by warp 0.
+// The shape and the A source are template parameters: the issue loop then holds no branch
+// and its descriptors stay in uniform registers, as in the library's kernels (with them as
+// run-time values one thread issued at half the rate).
+template <int M, int N, bool A_TMEM>
+__global__ void __launch_bounds__(64, 1)
+probe_mma_rate_kernel(int nissuers, int nmma, long long* cycles, int* ok,
+                      unsigned long long limit_ns) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  constexpr int kA = 16384, kB = 32768;  // 128 rows and 256 rows of 128 bytes
+  const uint32_t sb = smem_u32(smem);
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(smem + kA + kB);
+  const uint32_t bar0 = smem_u32(smem + kA + kB + 64), bar1 = bar0 + 8;
+  const uint32_t flag = smem_u32(smem + kA + kB + 128);
+  const int tid = threadIdx.x, warp = tid >> 5;
+  for (int i = tid; i < (kA + kB) / 4; i += blockDim.x) reinterpret_cast<uint32_t*>(smem)[i] = 0;
+  if (tid == 0) {
+    mbar_init(bar0, 1);
+    mbar_init(bar1, 1);
+    abort_set(flag, 0);
+    fence_barrier_init();
+  }
+  fence_proxy_async_smem();
+  if (warp == 0) {
+    tmem_alloc(smem_u32(tslot), kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tslot;
+  long long t0 = clock64();
+  if (warp < nissuers && (tid & 31) == 0) {
+    constexpr uint32_t idesc = idesc_bf16_f32(M, N, false, false);
+    const uint32_t a = sw128_lo(sb, 16), b = sw128_lo(sb + kA, 16);
+    const uint32_t d = tmem + warp * 128, at = tmem + 384;
+    const uint32_t bar = warp ? bar1 : bar0;
+    t0 = clock64();
+    for (int i = 0; i < nmma; ++i) {
+      if constexpr (A_TMEM)
+        mma_ts(d, at, sw128_at(b, (i & 3) * 32), idesc, i > 0);
+      else
+        mma_ss(d, sw128_at(a, (i & 3) * 32), sw128_at(b, (i & 3) * 32), idesc, i > 0);
+    }
+    mma_commit(bar);
+    const bool done = mbar_wait(bar, 0, flag, limit_ns);
+    const long long t1 = clock64();
+    if (warp == 0) cycles[blockIdx.x] = t1 - t0;
+    if (!done) atomicAnd(ok, 0);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
 }  // namespace
 
 extern "C" {
@@ -249,6 +315,52 @@ int probe_timeout(unsigned long long limit_ns, int* waited_ok_host) {
   cudaFree(dflag);
   cudaMemcpyToSymbol(ra::g_status, &zero, sizeof(int));
   return st;
+}
+
+
+// Average over one CTA per SM of the cycles per product of one SM (both issuers' products
+// counted), after one unmeasured launch.  N = 256 needs one issuer; two issuers need
+// N <= 128.  *ok_host = 1 if every wait completed.  Returns 0 or a CUDA error / -1.
+int probe_mma_rate(int M, int N, int a_tmem, int nissuers, int nmma, double* cycles_per_mma,
+                   int* ok_host) {
+  if (!(M == 64 || M == 128) || !(N == 32 || N == 64 || N == 128 || N == 256) ||
+      !(nissuers == 1 || nissuers == 2) || (nissuers == 2 && N > 128) || nmma < 1 ||
+      (a_tmem && M != 128))
+    return -1;
+  int dev = 0, nsm = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+  long long* cyc = nullptr;
+  int* ok = nullptr;
+  if (cudaMalloc(&cyc, nsm * sizeof(long long)) != cudaSuccess) return -2;
+  if (cudaMalloc(&ok, sizeof(int)) != cudaSuccess) return -2;
+  const int one = 1;
+  cudaMemcpy(ok, &one, sizeof(int), cudaMemcpyHostToDevice);
+  const int smem = 16384 + 32768 + 1024 + 256;
+  void (*k)(int, int, long long*, int*, unsigned long long) = nullptr;
+#define RA_PROBE_SHAPE(m, n)                                                    \
+  if (M == m && N == n)                                                         \
+    k = a_tmem ? probe_mma_rate_kernel<m, n, true> : probe_mma_rate_kernel<m, n, false>;
+  RA_PROBE_SHAPE(128, 32) RA_PROBE_SHAPE(128, 64) RA_PROBE_SHAPE(128, 128)
+  RA_PROBE_SHAPE(128, 256) RA_PROBE_SHAPE(64, 32) RA_PROBE_SHAPE(64, 64)
+  RA_PROBE_SHAPE(64, 128) RA_PROBE_SHAPE(64, 256)
+#undef RA_PROBE_SHAPE
+  cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  for (int rep = 0; rep < 2; ++rep)
+    k<<<nsm, 64, smem>>>(nissuers, nmma, cyc, ok, 2000000000ull);
+  int err = (int)cudaDeviceSynchronize();
+  if (err == 0) {
+    long long* h = new long long[nsm];
+    cudaMemcpy(h, cyc, nsm * sizeof(long long), cudaMemcpyDeviceToHost);
+    cudaMemcpy(ok_host, ok, sizeof(int), cudaMemcpyDeviceToHost);
+    double sum = 0.0;
+    for (int i = 0; i < nsm; ++i) sum += (double)h[i];
+    *cycles_per_mma = sum / nsm / ((double)nmma * nissuers);
+    delete[] h;
+  }
+  cudaFree(cyc);
+  cudaFree(ok);
+  return err;
 }
 
 }  // extern "C"

@@ -102,3 +102,28 @@ def test_turn_wait_gives_up(probe):
     assert st == 1 and ok == 0 and final == 4
     x = torch.ones(4, device="cuda")
     assert float(x.sum()) == 4.0
+
+
+def _mma_rate(probe, M, N, a_tmem=0, issuers=1, nmma=256):
+    cyc, ok = ctypes.c_double(), ctypes.c_int()
+    assert probe.probe_mma_rate(M, N, a_tmem, issuers, nmma, ctypes.byref(cyc),
+                                ctypes.byref(ok)) == 0
+    assert ok.value == 1
+    return cyc.value
+
+
+def test_mma_issue_rate(probe, capsys):
+    """Cycles one tcgen05.mma (K = 16) holds the tensor pipe, per shape: the products of the
+    backward (M = 128 x N = 64, M = 64 x N = 64, A from TMEM) against N = 128 and 256.  Every
+    product must complete; the time must grow with N past 128 (the probe measures executed
+    products).  The table is printed (pytest -s) for the design notes."""
+    shapes = [(128, 32, 0, 1), (128, 64, 0, 1), (128, 128, 0, 1), (128, 256, 0, 1),
+              (64, 64, 0, 1), (64, 128, 0, 1), (128, 64, 1, 1), (128, 128, 1, 1),
+              (128, 64, 0, 2), (128, 128, 0, 2)]
+    res = {sh: _mma_rate(probe, *sh) for sh in shapes}
+    with capsys.disabled():
+        for (M, N, at, iss), c in res.items():
+            print(f"M={M:3d} N={N:3d} A={'tmem' if at else 'smem'} issuers={iss}: "
+                  f"{c:6.1f} cycles per product (ideal {M * N * 16 / 4096:5.1f})")
+    assert res[(128, 256, 0, 1)] > 1.4 * res[(128, 128, 0, 1)]
+    assert all(c > 0 for c in res.values())

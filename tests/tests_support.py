@@ -17,4 +17,7 @@ def probe_lib():
                                ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int),
                                ctypes.POINTER(ctypes.c_uint)]
     lib.probe_turn.restype = ctypes.c_int
+    lib.probe_mma_rate.argtypes = [ctypes.c_int] * 5 + [ctypes.POINTER(ctypes.c_double),
+                                                        ctypes.POINTER(ctypes.c_int)]
+    lib.probe_mma_rate.restype = ctypes.c_int
     return lib
