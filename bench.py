@@ -384,7 +384,7 @@ def run_ours(args, rank, world, local_rank):
     top_ms, top_n = top_rec
     avg_ms = top_ms / max(1, top_n)
     sustained = ms_max >= SUSTAINED_REGION_MS
-    roof = roofline(w, top_name, avg_ms, pk, src, sustained)
+    roof = roofline(w, top_name, avg_ms, pk, src, sustained, det)
     value = whole_job_tflops(flops, args.steps, world, ms_max)
     total_kernel_ms = sum(v[0] for v in per_kernel.values())
     line = {
@@ -453,15 +453,17 @@ def kernel_roofline(w, kname, avg_ms, pk, sustained=False):
     return None
 
 
-def roofline(w, kname, avg_ms, pk, src, sustained=False):
-    """Algorithmic work of one launch of the dominant kernel over its measured duration."""
+def roofline(w, kname, avg_ms, pk, src, sustained=False, deterministic=False):
+    """Algorithmic work of one launch of the dominant kernel over its measured duration.
+    The DRAM traffic is the captured one for the default mode at the bench workload."""
     BH = w.B * w.H
     P = pair_count(w.n, w.causal)
     d, n = w.d, w.n
     tensor_kernels = {"attn_bwd_tc": 10.0 * d * P * BH, "attn_fwd_tc": 4.0 * d * P * BH}
     simt_kernels = {"attn_bwd_simt": 10.0 * d * P * BH, "attn_fwd_simt": 4.0 * d * P * BH,
                     "proj_rope_simt": 6.0 * n * d * d * BH, "dw_partial_simt": 6.0 * n * d * d * BH}
-    traffic = measured_traffic(kname) if w.name == DEFAULT_WORKLOAD else None
+    traffic = (measured_traffic(kname) if w.name == DEFAULT_WORKLOAD and not deterministic
+               else None)
     if kname in tensor_kernels:
         flop = tensor_kernels[kname]
         peak, kind = bf16_peak(pk, sustained)
