@@ -17,16 +17,20 @@
 //                                        reduce-add; the 1/sqrt(d) is applied when the
 //                                        accumulator is un-rotated, which keeps the drain warps'
 //                                        per-element work to a load and a store)
+//   at d = 64 instead, once per pair of query tiles i, i + 1:
+//   dQ~_i,i+1 = [gamma_i; gamma_i+1] K~  (the 128 queries on TMEM lanes, in columns of its own:
+//                                        a product with M = d = 64 holds the tensor pipe as
+//                                        long as one with M = 128)
 // so no n x n matrix ever leaves the chip.
 //
 // Definitions: "RoPE Attention kan bijna lineair worden getraind", Methodologie 1 (s, l,
 // beta, gamma) and 2 (gamma_1 = diag(s) beta, gamma_2 = s s^T beta).
 //
 // TMEM holds two step buffers of 128 columns, [S^T | beta^T] for query tiles i and i + 1
-// (i even in buffer 0), then dK~ and dV: while the softmax warps turn one buffer into P^T and
-// gamma^T, the tensor cores run the other buffer's products, and the next-but-one step's S^T
-// and beta^T are issued as soon as a buffer's products have completed and its dQ~^T has been
-// read out.
+// (i even in buffer 0), then dK~ and dV (and at d = 64 two 64-column buffers for the pair
+// products' dQ~): while the softmax warps turn one buffer into P^T and gamma^T, the tensor
+// cores run the other buffer's products, and the next-but-one step's S^T and beta^T are issued
+// as soon as a buffer's products have completed and (d = 128) its dQ~^T has been read out.
 //
 // Warp roles (480 threads): warps 0-7 softmax / gamma (two warpgroups over the same 128 key
 // rows, each taking half of the 64 query columns) and the epilogue (warps 0-3 dK, 4-7 dV),
