@@ -378,13 +378,22 @@ void finalize(const ra_problem* p, const Layout& L, void* ws, float* loss, int c
                                                     state);
 }
 
+// theta_k = base^(-2k/d) for k < d/2, in double precision.
+ra::simt::RopeTheta rope_theta(const ra_problem* p) {
+  ra::simt::RopeTheta th{};
+  const int half = p->d / 2;
+  for (int k = 0; k < half && k < ra::simt::kMaxHalf; ++k)
+    th.t[k] = std::pow(p->rope_base, -2.0 * (double)k / (double)p->d);
+  return th;
+}
+
 // RoPE table of the forward (grid-stride, a few blocks per SM).
 void rope_table(const ra_problem* p, const Layout& L, void* ws, cudaStream_t st) {
   const long long total = (long long)p->n * (p->d / 2);
   const long long want = (total + 255) / 256, cap = 8LL * num_sms();
   Launch l(K_ROPE_TABLE, st);
   ra::simt::rope_table_kernel<<<(unsigned)(want < cap ? want : cap), 256, 0, st>>>(
-      at<float2>(ws, L.rope), p->pos, p->n, p->d / 2, p->rope_base);
+      at<float2>(ws, L.rope), p->pos, p->n, p->d / 2, rope_theta(p));
 }
 
 // Gates of the backward.  With ws_holds_fwd the device decides from the workspace header:
@@ -413,7 +422,7 @@ void bwd_prep(const ra_problem* p, const Layout& L, const void* O, void* ws, con
                                      ra::simt::kThreads, 0, st>>>(
       (const T*)O, (const T*)p->E, at<TL>(ws, L.ell), at<float>(ws, L.delta),
       at<double>(ws, L.loss_part), p->n, p->d, (int)BH, at<float2>(ws, L.rope), p->pos,
-      p->rope_base, at<float4>(ws, L.dqt), BH * p->n * p->d / 4, g.recompute, g.zero,
+      rope_theta(p), at<float4>(ws, L.dqt), BH * p->n * p->d / 4, g.recompute, g.zero,
       p->deterministic ? at<unsigned>(ws, L.turn) : nullptr, BH * L.turn_stride);
 }
 
@@ -564,7 +573,8 @@ ra_status simt_input_grads(const ra_problem* p, const Layout& L, void* dA1, void
 
 template <int D>
 ra_status tc_weight_grads(const ra_problem* p, const Layout& L, float* dWQ, float* dWK,
-                          float* dWV, void* ws, ra::WsHeader* stamp, cudaStream_t st) {
+                          float* dWV, void* ws, ra::WsHeader* stamp,
+                          const ra::simt::LossSum& ls, cudaStream_t st) {
   using namespace ra::tc;
   using C = DwCfg<D>;
   const int n = p->n, BH = p->B * p->H, half = D / 2;
@@ -601,9 +611,11 @@ ra_status tc_weight_grads(const ra_problem* p, const Layout& L, float* dWQ, floa
   {
     size_t total = (size_t)3 * p->H * D * D;
     Launch l(K_DW_REDUCE, st);
-    ra::simt::dw_reduce_kernel<<<(unsigned)((total + 255) / 256), 256, 0, st>>>(
+    // with a loss to sum, one more block sums it and writes the header (no loss_finalize)
+    const unsigned blocks = (unsigned)((total + 255) / 256) + (ls.loss ? 1u : 0u);
+    ra::simt::dw_reduce_kernel<<<blocks, 256, 0, st>>>(
         at<float>(ws, L.dw_part), dWQ, dWK, dWV, p->H, D, L.nsplit, stamp, problem_tag(p),
-        ra::kWsValid);
+        ra::kWsValid, ls);
   }
   return launch_status();
 }
@@ -741,7 +753,8 @@ ra_status simt_bwd(const ra_problem* p, const void* O, const float* lse, float* 
     // header says so, written by the last launch of the call
     dw_reduce_kernel<<<(unsigned)((total + 255) / 256), 256, 0, st>>>(
         at<float>(ws, L.dw_part), dWQ, dWK, dWV, p->H, d, L.nsplit,
-        loss ? nullptr : at<ra::WsHeader>(ws, L.hdr), problem_tag(p), ra::kWsValid);
+        loss ? nullptr : at<ra::WsHeader>(ws, L.hdr), problem_tag(p), ra::kWsValid,
+        ra::simt::LossSum{});
   }
   if (loss) finalize(p, L, ws, loss, L.nparts_pre, g.recompute, ra::kWsValid, st);
   return launch_status();
@@ -760,12 +773,13 @@ ra_status tc_bwd(const ra_problem* p, const void* O, const float* lse, float* lo
   s = d == 128 ? tc_bwd_launch<128>(p, L, lse, ws, st) : tc_bwd_launch<64>(p, L, lse, ws, st);
   if (s != RA_OK) return s;
   // the workspace now holds this problem's intermediates and dQ~ is no longer zero: the header
-  // says so, written by the last launch of the call (loss_finalize when there is a loss to sum)
-  ra::WsHeader* stamp = loss ? nullptr : at<ra::WsHeader>(ws, L.hdr);
-  s = d == 128 ? tc_weight_grads<128>(p, L, dWQ, dWK, dWV, ws, stamp, st)
-               : tc_weight_grads<64>(p, L, dWQ, dWK, dWV, ws, stamp, st);
+  // says so, written by the last launch of the call, which also sums the loss
+  ra::WsHeader* stamp = at<ra::WsHeader>(ws, L.hdr);
+  const ra::simt::LossSum ls{at<double>(ws, L.loss_part), L.nparts_pre, L.nparts_fwd, loss,
+                             g.recompute};
+  s = d == 128 ? tc_weight_grads<128>(p, L, dWQ, dWK, dWV, ws, stamp, ls, st)
+               : tc_weight_grads<64>(p, L, dWQ, dWK, dWV, ws, stamp, ls, st);
   if (s != RA_OK) return s;
-  if (loss) finalize(p, L, ws, loss, L.nparts_pre, g.recompute, ra::kWsValid, st);
   return launch_status();
 }
 
@@ -792,11 +806,14 @@ ra_status tc_step(const ra_problem* p, void* O, float* lse, float* loss, float* 
     return RA_ERR_CUDA;
   s = d == 128 ? tc_bwd_launch<128>(p, L, lse, ws, st) : tc_bwd_launch<64>(p, L, lse, ws, st);
   if (s != RA_OK) return s;
-  ra::WsHeader* stamp = loss ? nullptr : at<ra::WsHeader>(ws, L.hdr);
-  s = d == 128 ? tc_weight_grads<128>(p, L, dWQ, dWK, dWV, ws, stamp, st)
-               : tc_weight_grads<64>(p, L, dWQ, dWK, dWV, ws, stamp, st);
+  // the last launch sums the loss (the forward's partials) and writes the header
+  const ra::simt::LossSum ls{at<double>(ws, L.loss_part), L.nparts_fwd, L.nparts_fwd, loss,
+                             none};
+  s = d == 128 ? tc_weight_grads<128>(p, L, dWQ, dWK, dWV, ws, at<ra::WsHeader>(ws, L.hdr), ls,
+                                      st)
+               : tc_weight_grads<64>(p, L, dWQ, dWK, dWV, ws, at<ra::WsHeader>(ws, L.hdr), ls,
+                                     st);
   if (s != RA_OK) return s;
-  if (loss) finalize(p, L, ws, loss, L.nparts_fwd, none, ra::kWsValid, st);
   return launch_status();
 }
 
@@ -911,7 +928,7 @@ ra_status approx_step(const ra_problem* p, void* O, float* loss, float* dWQ, flo
     const long long want = (total + 255) / 256, cap = 8LL * num_sms();
     Launch l(K_ROPE_TABLE, st);
     ra::simt::rope_table_kernel<<<(unsigned)(want < cap ? want : cap), 256, 0, st>>>(
-        tab, p->pos, n, D / 2, p->rope_base);
+        tab, p->pos, n, D / 2, rope_theta(p));
   }
   {
     using namespace ra::simt;
@@ -987,7 +1004,8 @@ ra_status approx_step(const ra_problem* p, void* O, float* loss, float* dWQ, flo
     size_t total = (size_t)3 * p->H * D * D;
     Launch l(K_DW_REDUCE, st);
     dw_reduce_kernel<<<(unsigned)((total + 255) / 256), 256, 0, st>>>(
-        at<float>(ws, L.dw_part), dWQ, dWK, dWV, p->H, D, L.nsplit, nullptr, 0, 0u);
+        at<float>(ws, L.dw_part), dWQ, dWK, dWV, p->H, D, L.nsplit, nullptr, 0, 0u,
+        ra::simt::LossSum{});
   }
   if (loss) {
     Launch l(K_LOSS, st);

@@ -14,33 +14,41 @@ constexpr int kRows = 32;      // query (or key) rows per block
 constexpr int kThreads = 256;  // 8 threads per row
 
 // ---------------------------------------------------------------------------------------
-// RoPE table: tab[i][k] = (cos, sin)(pos_i * base^(-2k/d)), angle and sin/cos in fp64.
-// Grid-stride over the n * half entries; each block first puts theta_k = base^(-2k/d) for the
-// half <= 64 frequencies in shared memory, so pow runs once per block and frequency.
+// RoPE table: tab[i][k] = (cos, sin)(pos_i * base^(-2k/d)), grid-stride over the n * half
+// entries; the half <= 64 frequencies come from the host.
 // ---------------------------------------------------------------------------------------
 constexpr int kMaxHalf = 64;
 
+// theta_k = base^(-2k/d), k < d/2, computed on the host in double precision.
+struct RopeTheta {
+  double t[kMaxHalf];
+};
+
+// (cos, sin) of pos_i theta_k for every row i and pair k.  The angle (up to about 1.3e5 rad at
+// n = 131072) is formed and reduced to [-pi, pi] in double precision (2 pi as a double leaves
+// an error of m * 2.4e-16 rad after m turns, far below what the fp32 table resolves); the sine
+// and cosine of the reduced angle are then taken in single precision (sincosf), which on that
+// range is accurate to a few fp32 ulps.
 __device__ __forceinline__ void rope_table_fill(float2* __restrict__ tab,
                                                 const int32_t* __restrict__ pos, int n, int half,
-                                                double base) {
-  __shared__ double theta[kMaxHalf];
-  for (int k = threadIdx.x; k < half; k += blockDim.x)
-    theta[k] = pow(base, -2.0 * (double)k / (double)(2 * half));
-  __syncthreads();
+                                                const RopeTheta& th) {
+  constexpr double kTwoPi = 6.283185307179586, kInvTwoPi = 0.15915494309189535;
   const long long total = (long long)n * half;
   for (long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
        idx += (long long)gridDim.x * blockDim.x) {
     const int i = (int)(idx / half), k = (int)(idx - (long long)i * half);
     const double p = pos ? (double)pos[i] : (double)i;
-    double sn, cs;
-    sincos(p * theta[k], &sn, &cs);
-    tab[idx] = make_float2((float)cs, (float)sn);
+    const double a = p * th.t[k];
+    const double r = a - rint(a * kInvTwoPi) * kTwoPi;
+    float sn, cs;
+    sincosf(static_cast<float>(r), &sn, &cs);
+    tab[idx] = make_float2(cs, sn);
   }
 }
 
 __global__ void rope_table_kernel(float2* __restrict__ tab, const int32_t* __restrict__ pos,
-                                  int n, int half, double base) {
-  rope_table_fill(tab, pos, n, half, base);
+                                  int n, int half, const RopeTheta th) {
+  rope_table_fill(tab, pos, n, half, th);
 }
 
 // ---------------------------------------------------------------------------------------
@@ -264,13 +272,13 @@ template <class T, class TL>
 __global__ void __launch_bounds__(kThreads)
 bwd_prep_kernel(const T* __restrict__ O, const T* __restrict__ E, TL* __restrict__ ell,
                 float* __restrict__ delta, double* __restrict__ loss_part, int n, int d, int BH,
-                float2* __restrict__ tab, const int32_t* __restrict__ pos, double base,
+                float2* __restrict__ tab, const int32_t* __restrict__ pos, const RopeTheta th,
                 float4* __restrict__ dq, long long n4, WsGate recompute, WsGate zero,
                 unsigned* __restrict__ turn, long long nturn) {
   __shared__ double red[kThreads / 32];
   const bool rec = !gate_skip(recompute), zer = !gate_skip(zero);
   if (rec) {
-    rope_table_fill(tab, pos, n, d / 2, base);
+    rope_table_fill(tab, pos, n, d / 2, th);
     const int nrb = (n + kRows - 1) / kRows;
     const long long nvb = (long long)nrb * BH;
     for (long long vb = blockIdx.x; vb < nvb; vb += gridDim.x)
@@ -493,16 +501,66 @@ dw_partial_kernel(const TA* __restrict__ A1, const TA* __restrict__ A2, const TA
     for (int c = 0; c < sub; ++c) dst[(size_t)(ti + a) * d + tj + c] = acc[a][c];
 }
 
-// dW[z][h] = sum over splits (fixed order) of part[z][h][split].
-// When `stamp` is given (a backward without a loss to sum, so no loss_finalize follows),
-// thread 0 also writes the workspace header (stamp_tag, stamp_state).
+// Sum of the loss partials part[0 .. count) in a fixed order that does not depend on the block
+// size: 1024 virtual lanes, lane v adding partials v, v + 1024, ... in four interleaved chains,
+// then a pairwise tree over the lanes.  One block of blockDim.x threads (a divisor of 1024)
+// computes it; red holds 1024 doubles of shared memory.  The result is red[0].
+__device__ __forceinline__ void loss_sum_fixed(const double* __restrict__ part, int count,
+                                               double* red) {
+  constexpr int V = 1024;
+  for (int v = threadIdx.x; v < V; v += blockDim.x) {
+    double s0 = 0.0, s1 = 0.0, s2 = 0.0, s3 = 0.0;
+    int i = v;
+    for (; i + 3 * V < count; i += 4 * V) {
+      s0 += part[i];
+      s1 += part[i + V];
+      s2 += part[i + 2 * V];
+      s3 += part[i + 3 * V];
+    }
+    for (; i < count; i += V) s0 += part[i];
+    red[v] = (s0 + s1) + (s2 + s3);
+  }
+  __syncthreads();
+  for (int w = V / 2; w > 0; w >>= 1) {
+    for (int v = threadIdx.x; v < w; v += blockDim.x) red[v] += red[v + w];
+    __syncthreads();
+  }
+}
+
+// The loss of a call, summed by the last launch that needs it.  `count` partials belong to
+// this call; when `gate` finds the backward's recomputation skipped, the forward's `count_kept`
+// ones are summed.
+struct LossSum {
+  const double* part;
+  int count, count_kept;
+  float* loss;  // null: no loss to sum
+  WsGate gate;
+};
+
+// dW_z[h] = sum over the nsplit row-range partials in a fixed order (fp64), one thread per
+// output element.  With a loss to sum, one more block (block 0, so that it runs beside the
+// others rather than after them) sums it and writes the workspace header; otherwise thread 0
+// writes the header (stamp non-null).
 __global__ void dw_reduce_kernel(const float* __restrict__ part, float* __restrict__ dWQ,
                                  float* __restrict__ dWK, float* __restrict__ dWV, int H, int d,
                                  int nsplit, WsHeader* stamp, unsigned long long stamp_tag,
-                                 unsigned int stamp_state) {
+                                 unsigned int stamp_state, LossSum ls) {
+  if (ls.loss && blockIdx.x == 0) {
+    __shared__ double red[1024];
+    const int count = gate_skip(ls.gate) ? ls.count_kept : ls.count;
+    __syncthreads();  // every thread has read the header before thread 0 rewrites it
+    if (stamp && threadIdx.x == 0) {
+      stamp->tag = stamp_tag;
+      stamp->state = stamp_state;
+      stamp->magic = kWsMagic;
+    }
+    loss_sum_fixed(ls.part, count, red);
+    if (threadIdx.x == 0) *ls.loss = (float)red[0];
+    return;
+  }
   const size_t dd = (size_t)d * d;
-  const size_t idx = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (stamp && idx == 0) {
+  const size_t idx = (size_t)(blockIdx.x - (ls.loss ? 1 : 0)) * blockDim.x + threadIdx.x;
+  if (stamp && !ls.loss && idx == 0) {
     stamp->tag = stamp_tag;
     stamp->state = stamp_state;
     stamp->magic = kWsMagic;
@@ -526,8 +584,8 @@ __global__ void dw_reduce_kernel(const float* __restrict__ part, float* __restri
 __global__ void loss_finalize_kernel(const double* __restrict__ part, int count, int count_kept,
                                      float* __restrict__ loss, WsGate gate, WsHeader* stamp,
                                      unsigned long long stamp_tag, unsigned int stamp_state) {
-  // fixed summation order for a given count and block size (deterministic); four
-  // independent partial sums per thread keep the loads in flight
+  // fixed summation order for a given count, whatever the block size (deterministic, and the
+  // same as the loss block of dw_reduce_kernel)
   __shared__ double red[1024];
   if (gate_skip(gate)) count = count_kept;
   __syncthreads();  // every thread has read the header before thread 0 rewrites it
@@ -537,22 +595,7 @@ __global__ void loss_finalize_kernel(const double* __restrict__ part, int count,
     stamp->magic = kWsMagic;
   }
   if (!loss) return;
-  double s0 = 0.0, s1 = 0.0, s2 = 0.0, s3 = 0.0;
-  const int stride = blockDim.x;
-  int i = threadIdx.x;
-  for (; i + 3 * stride < count; i += 4 * stride) {
-    s0 += part[i];
-    s1 += part[i + stride];
-    s2 += part[i + 2 * stride];
-    s3 += part[i + 3 * stride];
-  }
-  for (; i < count; i += stride) s0 += part[i];
-  red[threadIdx.x] = (s0 + s1) + (s2 + s3);
-  __syncthreads();
-  for (int w = blockDim.x / 2; w > 0; w >>= 1) {
-    if ((int)threadIdx.x < w) red[threadIdx.x] += red[threadIdx.x + w];
-    __syncthreads();
-  }
+  loss_sum_fixed(part, count, red);
   if (threadIdx.x == 0) *loss = (float)red[0];
 }
 
