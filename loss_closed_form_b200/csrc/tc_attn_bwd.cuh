@@ -250,9 +250,10 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     // tensor pipe takes the product, so with one thread a wait for one chain (the drain
     // freeing beta^T's columns) also held the other (the next step's products).
     //   step i, buffer b = i % 2:  S^T_i once dV and dK of step i - 2 have read P^T, gamma^T
-    //   over its columns; beta^T_i once the drain has read dQ~^T_i-2 over its columns;
-    //   dV, dK (P^T, gamma^T from TMEM) then dQ~^T_i (over the beta^T columns, which the
-    //   softmax warps have read) once P^T_i, gamma^T_i are written.
+    //   over its columns; beta^T_i (d = 128) once the drain has read dQ~^T_i-2 over its
+    //   columns; dV, dK (P^T, gamma^T from TMEM) then dQ~^T_i (over the beta^T columns, which
+    //   the softmax warps have read) once P^T_i, gamma^T_i are written.  At d = 64 the pair
+    //   products' dQ~ has columns of its own, so beta^T_i waits only for its query tile.
     // Both poll their barriers: a suspended wait resumes a few hundred cycles after the phase
     // completes, on the chain every step waits for.
     if (lane == 0) {
